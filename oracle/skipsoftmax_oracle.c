@@ -1,0 +1,388 @@
+/*
+ * Plain fp64 CPU oracle for Skip Softmax attention (prefill and decode).
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the product path may include, link or
+ * call this file; it exists so that tests, the smoke check and the bench's CPU
+ * baseline can check the CUDA kernels against an obviously correct program.
+ * It shares no code, header, table or constant with the CUDA path.
+ *
+ * What it computes (source: "Accelerating Long-Context Inference with Skip
+ * Softmax in NVIDIA TensorRT-LLM", Key Points and Detailed Analysis):
+ *   attention scores S = Q K^T / sqrt(d) are visited one key block (tile) at a
+ *   time, in ascending key order.  For each visited tile j the local maximum
+ *   of every query row, mt_r = max_{k in tile} s_rk, is compared with the
+ *   running row maximum m_r minus the threshold tau.  If every row of the row
+ *   block has mt_r < m_r - tau (strict), the whole tile is skipped: none of its
+ *   exponentials is formed and none of its values is accumulated.  Otherwise
+ *   the usual online-softmax update runs:
+ *        m' = max(m, mt);   l = l e^{m-m'} + sum_k e^{s-m'};
+ *        acc = acc e^{m-m'} + sum_k e^{s-m'} v_k;   m = m'.
+ *   The output row is acc / l.  (The page's comparison value is garbled in
+ *   the transcript; it is read as m_i - tau, the running maximum minus the
+ *   threshold the page calls Tau.)
+ *
+ * Conventions fixed where the page is silent:
+ *   - causal attention is top-left aligned: query i sees keys k <= i; tiles
+ *     whose first key lies beyond the last row of the row block are not
+ *     visited at all (mask value 2);
+ *   - a row whose running max is still -inf cannot be skipped (tile 0 is
+ *     therefore always kept); a row whose tile max is -inf (fully masked in
+ *     this tile) does not prevent skipping;
+ *   - tau >= 0, tau = +inf means exact attention;
+ *   - decode: the rows of the test are the g query heads that share one KV
+ *     head; the key range is cut into splits of Ls keys, each split runs the
+ *     tile loop with its own running max starting at -inf, and the split
+ *     results are merged exactly (log-sum-exp).
+ *
+ * Every floating-point quantity is fp64; inputs are bf16 bit patterns that are
+ * widened exactly.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_OK 0
+#define ORACLE_BAD_ARG 1
+#define ORACLE_NO_MEMORY 2
+
+/* bf16 -> fp64: a bf16 value is the top half of an IEEE fp32 word. */
+static double widen_bf16(uint16_t bits)
+{
+    uint32_t w = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &w, sizeof f);
+    return (double)f;
+}
+
+static double dot_widened(const uint16_t *a, const uint16_t *b, int d)
+{
+    double s = 0.0;
+    for (int t = 0; t < d; ++t)
+        s += widen_bf16(a[t]) * widen_bf16(b[t]);
+    return s;
+}
+
+/* Contribution of one row to the tile margin  max_r (mt_r - m_r + tau).
+ * The tile is skipped iff the maximum over rows is < 0.                   */
+static double row_margin(double mt, double m, double tau)
+{
+    if (m == -INFINITY) return INFINITY;     /* nothing seen yet: never skippable */
+    if (mt == -INFINITY) return -INFINITY;   /* row fully masked in this tile      */
+    return mt - m + tau;                     /* tau = +inf gives +inf               */
+}
+
+/* ------------------------------------------------------------------------- */
+/* Prefill                                                                   */
+/* ------------------------------------------------------------------------- */
+
+typedef struct {
+    const uint16_t *Q, *K, *V;
+    int B, Hq, Hkv, N, d, causal, Br, Bc;
+    double tau;
+    double *O, *O_exact, *margin, *pskip;
+    uint8_t *mask;
+} prefill_args;
+
+/* One row block: rows [r0, r1) of query head h in batch b. */
+static int prefill_row_block(const prefill_args *a, int b, int h, int rb)
+{
+    const int N = a->N, d = a->d, Br = a->Br, Bc = a->Bc;
+    const int g = a->Hq / a->Hkv;
+    const int kvh = h / g;                       /* query head h reads KV head floor(h/g) */
+    const int n_rb = (N + Br - 1) / Br;
+    const int n_tiles = (N + Bc - 1) / Bc;
+    const int r0 = rb * Br;
+    const int r1 = (r0 + Br < N) ? r0 + Br : N;
+    const int nr = r1 - r0;
+    const double inv_sqrt_d = 1.0 / sqrt((double)d);
+
+    const uint16_t *q = a->Q + ((size_t)(b * a->Hq + h) * N) * d;
+    const uint16_t *k = a->K + ((size_t)(b * a->Hkv + kvh) * N) * d;
+    const uint16_t *v = a->V + ((size_t)(b * a->Hkv + kvh) * N) * d;
+
+    double *m = malloc(sizeof(double) * nr);
+    double *l = malloc(sizeof(double) * nr);
+    double *acc = calloc((size_t)nr * d, sizeof(double));
+    double *s = malloc(sizeof(double) * (size_t)nr * Bc);
+    double *mt = malloc(sizeof(double) * nr);
+    uint8_t *skipped = calloc(n_tiles, 1);
+    if (!m || !l || !acc || !s || !mt || !skipped) {
+        free(m); free(l); free(acc); free(s); free(mt); free(skipped);
+        return ORACLE_NO_MEMORY;
+    }
+    for (int r = 0; r < nr; ++r) { m[r] = -INFINITY; l[r] = 0.0; }
+
+    const size_t tile_base = (((size_t)b * a->Hq + h) * n_rb + rb) * n_tiles;
+
+    for (int j = 0; j < n_tiles; ++j) {
+        const int c0 = j * Bc;
+        const int c1 = (c0 + Bc < N) ? c0 + Bc : N;
+        if (a->causal && c0 > r1 - 1) {          /* tile lies wholly above the diagonal */
+            if (a->mask) a->mask[tile_base + j] = 2;
+            if (a->margin) a->margin[tile_base + j] = NAN;
+            continue;
+        }
+        /* scores of this tile and the local (tile) maximum of every row */
+        for (int r = 0; r < nr; ++r) {
+            const int qi = r0 + r;
+            mt[r] = -INFINITY;
+            for (int c = c0; c < c1; ++c) {
+                double x;
+                if (a->causal && c > qi) x = -INFINITY;
+                else x = dot_widened(q + (size_t)qi * d, k + (size_t)c * d, d) * inv_sqrt_d;
+                s[(size_t)r * Bc + (c - c0)] = x;
+                if (x > mt[r]) mt[r] = x;
+            }
+        }
+        /* the block-skip test */
+        double margin = -INFINITY;
+        for (int r = 0; r < nr; ++r) {
+            double x = row_margin(mt[r], m[r], a->tau);
+            if (x > margin) margin = x;
+        }
+        const int skip = margin < 0.0;
+        if (a->mask) a->mask[tile_base + j] = (uint8_t)skip;
+        if (a->margin) a->margin[tile_base + j] = margin;
+        if (skip) { skipped[j] = 1; continue; }
+
+        /* online-softmax update with this tile */
+        for (int r = 0; r < nr; ++r) {
+            const double m_new = (mt[r] > m[r]) ? mt[r] : m[r];
+            if (m_new == -INFINITY) continue;    /* row has seen no visible key yet */
+            const double alpha = (m[r] == -INFINITY) ? 0.0 : exp(m[r] - m_new);
+            l[r] *= alpha;
+            double *ar = acc + (size_t)r * d;
+            for (int t = 0; t < d; ++t) ar[t] *= alpha;
+            for (int c = c0; c < c1; ++c) {
+                const double x = s[(size_t)r * Bc + (c - c0)];
+                if (x == -INFINITY) continue;
+                const double p = exp(x - m_new);
+                l[r] += p;
+                const uint16_t *vc = v + (size_t)c * d;
+                for (int t = 0; t < d; ++t) ar[t] += p * widen_bf16(vc[t]);
+            }
+            m[r] = m_new;
+        }
+    }
+
+    for (int r = 0; r < nr; ++r) {
+        double *o = a->O + ((size_t)(b * a->Hq + h) * N + r0 + r) * d;
+        for (int t = 0; t < d; ++t) o[t] = acc[(size_t)r * d + t] / l[r];
+    }
+
+    /* exact attention (every visible key) and the probability mass the skip
+     * removed, both straight from the softmax definition                     */
+    if (a->O_exact || a->pskip) {
+        double *w = malloc(sizeof(double) * N);
+        double *ex = malloc(sizeof(double) * d);
+        if (!w || !ex) { free(w); free(ex); free(m); free(l); free(acc); free(s); free(mt); free(skipped); return ORACLE_NO_MEMORY; }
+        for (int r = 0; r < nr; ++r) {
+            const int qi = r0 + r;
+            const int kend = a->causal ? qi + 1 : N;
+            double M = -INFINITY;
+            for (int c = 0; c < kend; ++c) {
+                w[c] = dot_widened(q + (size_t)qi * d, k + (size_t)c * d, d) * inv_sqrt_d;
+                if (w[c] > M) M = w[c];
+            }
+            double total = 0.0, lost = 0.0;
+            for (int t = 0; t < d; ++t) ex[t] = 0.0;
+            for (int c = 0; c < kend; ++c) {
+                const double p = exp(w[c] - M);
+                total += p;
+                if (skipped[c / Bc]) lost += p;
+                const uint16_t *vc = v + (size_t)c * d;
+                for (int t = 0; t < d; ++t) ex[t] += p * widen_bf16(vc[t]);
+            }
+            const size_t row = (size_t)(b * a->Hq + h) * N + qi;
+            if (a->O_exact)
+                for (int t = 0; t < d; ++t) a->O_exact[row * d + t] = ex[t] / total;
+            if (a->pskip) a->pskip[row] = lost / total;
+        }
+        free(w); free(ex);
+    }
+
+    free(m); free(l); free(acc); free(s); free(mt); free(skipped);
+    return ORACLE_OK;
+}
+
+/*
+ * Q [B,Hq,N,d], K/V [B,Hkv,N,d] bf16 bits, contiguous, d fastest.
+ * units: NULL for every row block, else n_units triples (b, h, rb).
+ * O [B,Hq,N,d] fp64 (required).  Optional (may be NULL):
+ *   O_exact [B,Hq,N,d]      exact attention (no skipping)
+ *   mask    [B,Hq,nRB,nT]   0 kept, 1 skipped, 2 not visited (causal)
+ *   margin  [B,Hq,nRB,nT]   max_r (mt_r - m_r + tau), NaN if not visited
+ *   pskip   [B,Hq,N]        softmax probability mass in skipped tiles
+ * Only the entries belonging to the computed row blocks are written.
+ */
+int oracle_prefill(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
+                   int B, int Hq, int Hkv, int N, int d, int causal, double tau,
+                   int Br, int Bc, const int32_t *units, int64_t n_units,
+                   double *O, double *O_exact, uint8_t *mask, double *margin,
+                   double *pskip, int nthreads)
+{
+    if (!Q || !K || !V || !O) return ORACLE_BAD_ARG;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0 || d <= 0 || Br <= 0 || Bc <= 0) return ORACLE_BAD_ARG;
+    if (Hq % Hkv != 0) return ORACLE_BAD_ARG;
+    if (isnan(tau) || tau < 0.0) return ORACLE_BAD_ARG;
+
+    prefill_args a = {Q, K, V, B, Hq, Hkv, N, d, causal, Br, Bc, tau, O, O_exact, margin, pskip, mask};
+    const int n_rb = (N + Br - 1) / Br;
+    const int64_t total = units ? n_units : (int64_t)B * Hq * n_rb;
+    int status = ORACLE_OK;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t u = 0; u < total; ++u) {
+        int b, h, rb;
+        if (units) { b = units[3 * u]; h = units[3 * u + 1]; rb = units[3 * u + 2]; }
+        else { rb = (int)(u % n_rb); h = (int)((u / n_rb) % Hq); b = (int)(u / ((int64_t)n_rb * Hq)); }
+        int st;
+        if (b < 0 || b >= B || h < 0 || h >= Hq || rb < 0 || rb >= n_rb) st = ORACLE_BAD_ARG;
+        else st = prefill_row_block(&a, b, h, rb);
+        if (st != ORACLE_OK) {
+#pragma omp critical
+            status = st;
+        }
+    }
+    return status;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Decode                                                                    */
+/* ------------------------------------------------------------------------- */
+
+/*
+ * q [B,Hq,d]; K/V [B,Hkv,L,d]; one query token per (batch, query head) that
+ * attends to all L cached keys.  Rows of the skip test: the g = Hq/Hkv query
+ * heads of one KV head.  Splits of Ls keys, tiles of Bt keys inside a split.
+ * o [B,Hq,d] fp64.  Optional: o_exact [B,Hq,d]; mask/margin [B,Hkv,ceil(L/Bt)]
+ * (tiles are numbered globally: tile j covers keys [j*Bt, (j+1)*Bt) cut at the
+ * split end, so Ls must be a multiple of Bt); pskip [B,Hq].
+ */
+int oracle_decode(const uint16_t *q, const uint16_t *K, const uint16_t *V,
+                  int B, int Hq, int Hkv, int L, int d, double tau, int Ls, int Bt,
+                  double *o, double *o_exact, uint8_t *mask, double *margin,
+                  double *pskip, int nthreads)
+{
+    if (!q || !K || !V || !o) return ORACLE_BAD_ARG;
+    if (B <= 0 || Hq <= 0 || Hkv <= 0 || L <= 0 || d <= 0 || Ls <= 0 || Bt <= 0) return ORACLE_BAD_ARG;
+    if (Hq % Hkv != 0 || Ls % Bt != 0) return ORACLE_BAD_ARG;
+    if (isnan(tau) || tau < 0.0) return ORACLE_BAD_ARG;
+    const int g = Hq / Hkv;
+    const int n_tiles = (L + Bt - 1) / Bt;
+    const int n_splits = (L + Ls - 1) / Ls;
+    const double inv_sqrt_d = 1.0 / sqrt((double)d);
+    int status = ORACLE_OK;
+#ifdef _OPENMP
+    if (nthreads > 0) omp_set_num_threads(nthreads);
+#else
+    (void)nthreads;
+#endif
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t grp = 0; grp < (int64_t)B * Hkv; ++grp) {
+        const int b = (int)(grp / Hkv), kvh = (int)(grp % Hkv);
+        const uint16_t *k = K + ((size_t)(b * Hkv + kvh) * L) * d;
+        const uint16_t *v = V + ((size_t)(b * Hkv + kvh) * L) * d;
+        double *s = malloc(sizeof(double) * (size_t)L * g);       /* all scores, [key][row] */
+        double *m = malloc(sizeof(double) * g), *l = malloc(sizeof(double) * g);
+        double *acc = malloc(sizeof(double) * (size_t)g * d);
+        double *sm = malloc(sizeof(double) * (size_t)n_splits * g);   /* per-split max   */
+        double *sl = malloc(sizeof(double) * (size_t)n_splits * g);   /* per-split sum   */
+        double *sa = malloc(sizeof(double) * (size_t)n_splits * g * d);/* per-split acc  */
+        double *mt = malloc(sizeof(double) * g);
+        uint8_t *skipped = calloc(n_tiles, 1);
+        if (!s || !m || !l || !acc || !sm || !sl || !sa || !mt || !skipped) {
+#pragma omp critical
+            status = ORACLE_NO_MEMORY;
+            free(s); free(m); free(l); free(acc); free(sm); free(sl); free(sa); free(mt); free(skipped);
+            continue;
+        }
+        for (int c = 0; c < L; ++c)
+            for (int r = 0; r < g; ++r) {
+                const uint16_t *qr = q + ((size_t)b * Hq + (size_t)kvh * g + r) * d;
+                s[(size_t)c * g + r] = dot_widened(qr, k + (size_t)c * d, d) * inv_sqrt_d;
+            }
+        for (int sp = 0; sp < n_splits; ++sp) {
+            const int k0 = sp * Ls, k1 = (k0 + Ls < L) ? k0 + Ls : L;
+            for (int r = 0; r < g; ++r) { m[r] = -INFINITY; l[r] = 0.0; }
+            for (size_t t = 0; t < (size_t)g * d; ++t) acc[t] = 0.0;
+            for (int c0 = k0; c0 < k1; c0 += Bt) {
+                const int c1 = (c0 + Bt < k1) ? c0 + Bt : k1;
+                const int j = c0 / Bt;
+                double margin_j = -INFINITY;
+                for (int r = 0; r < g; ++r) {
+                    mt[r] = -INFINITY;
+                    for (int c = c0; c < c1; ++c)
+                        if (s[(size_t)c * g + r] > mt[r]) mt[r] = s[(size_t)c * g + r];
+                    double x = row_margin(mt[r], m[r], tau);
+                    if (x > margin_j) margin_j = x;
+                }
+                const int skip = margin_j < 0.0;
+                const size_t ti = (size_t)(b * Hkv + kvh) * n_tiles + j;
+                if (mask) mask[ti] = (uint8_t)skip;
+                if (margin) margin[ti] = margin_j;
+                if (skip) { skipped[j] = 1; continue; }
+                for (int r = 0; r < g; ++r) {
+                    const double m_new = (mt[r] > m[r]) ? mt[r] : m[r];
+                    const double alpha = (m[r] == -INFINITY) ? 0.0 : exp(m[r] - m_new);
+                    l[r] *= alpha;
+                    for (int t = 0; t < d; ++t) acc[(size_t)r * d + t] *= alpha;
+                    for (int c = c0; c < c1; ++c) {
+                        const double p = exp(s[(size_t)c * g + r] - m_new);
+                        l[r] += p;
+                        for (int t = 0; t < d; ++t) acc[(size_t)r * d + t] += p * widen_bf16(v[(size_t)c * d + t]);
+                    }
+                    m[r] = m_new;
+                }
+            }
+            for (int r = 0; r < g; ++r) {
+                sm[(size_t)sp * g + r] = m[r];
+                sl[(size_t)sp * g + r] = l[r];
+                for (int t = 0; t < d; ++t) sa[((size_t)sp * g + r) * d + t] = acc[(size_t)r * d + t];
+            }
+        }
+        /* exact merge of the splits: rescale each to the common maximum */
+        for (int r = 0; r < g; ++r) {
+            double M = -INFINITY;
+            for (int sp = 0; sp < n_splits; ++sp)
+                if (sm[(size_t)sp * g + r] > M) M = sm[(size_t)sp * g + r];
+            double den = 0.0;
+            double *orow = o + ((size_t)b * Hq + (size_t)kvh * g + r) * d;
+            for (int t = 0; t < d; ++t) orow[t] = 0.0;
+            for (int sp = 0; sp < n_splits; ++sp) {
+                const double w = exp(sm[(size_t)sp * g + r] - M);
+                den += w * sl[(size_t)sp * g + r];
+                for (int t = 0; t < d; ++t) orow[t] += w * sa[((size_t)sp * g + r) * d + t];
+            }
+            for (int t = 0; t < d; ++t) orow[t] /= den;
+        }
+        /* exact attention and skipped probability mass, from the definition */
+        if (o_exact || pskip) {
+            for (int r = 0; r < g; ++r) {
+                double M = -INFINITY;
+                for (int c = 0; c < L; ++c) if (s[(size_t)c * g + r] > M) M = s[(size_t)c * g + r];
+                double total = 0.0, lost = 0.0;
+                for (int t = 0; t < d; ++t) acc[t] = 0.0;
+                for (int c = 0; c < L; ++c) {
+                    const double p = exp(s[(size_t)c * g + r] - M);
+                    total += p;
+                    if (skipped[c / Bt]) lost += p;
+                    for (int t = 0; t < d; ++t) acc[t] += p * widen_bf16(v[(size_t)c * d + t]);
+                }
+                const size_t row = (size_t)b * Hq + (size_t)kvh * g + r;
+                if (o_exact) for (int t = 0; t < d; ++t) o_exact[row * d + t] = acc[t] / total;
+                if (pskip) pskip[row] = lost / total;
+            }
+        }
+        free(s); free(m); free(l); free(acc); free(sm); free(sl); free(sa); free(mt); free(skipped);
+    }
+    return status;
+}

@@ -1,0 +1,411 @@
+"""Pins for the fp64 CPU oracle: what the mathematics and the pages fix.
+
+The oracle is only trusted after it is pinned to something other than
+itself.  Each pin below is written against the definition of attention
+(brute force on tiny inputs), a closed form, an invariant, or the hand-built
+two-tile example in ``tests/golden/two_tile_example.txt``.  The rule pinned
+is the one of "Accelerating Long-Context Inference with Skip Softmax in NVIDIA
+TensorRT-LLM" (Key Points; Detailed Analysis).
+
+Every pin takes ``lib`` (None for the real oracle, or the path of a variant
+built by ``test_oracle_mutants.py``) so that the same pins can be shown to
+catch planted mistakes.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from block_skipping_softmax_b200 import inputs
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "two_tile_example.txt")
+PINS = []
+
+
+def pin(fn):
+    PINS.append(fn)
+    return fn
+
+
+# ----------------------------------------------------------------------------
+# independent numpy helpers (fp64, whole score matrix, no tiling)
+# ----------------------------------------------------------------------------
+
+def f64(x):
+    return x.float().double().numpy() if isinstance(x, torch.Tensor) else np.asarray(x, np.float64)
+
+
+def scores(Q, K, causal):
+    """S[b,h,i,k] = q_i . k_k / sqrt(d), -inf above the diagonal when causal."""
+    q, k = f64(Q), f64(K)
+    g = q.shape[1] // k.shape[1]
+    k = np.repeat(k, g, axis=1)                       # head h reads KV head h // g
+    s = np.einsum("bhid,bhkd->bhik", q, k) / math.sqrt(q.shape[-1])
+    if causal:
+        n = s.shape[-1]
+        s = np.where(np.triu(np.ones((n, n), bool), 1), -np.inf, s)
+    return s
+
+
+def softmax_av(s, V, keep=None):
+    """softmax over the last axis (optionally restricted by a boolean keep) times V."""
+    g = s.shape[1] // V.shape[1]
+    v = np.repeat(f64(V), g, axis=1)
+    if keep is not None:
+        s = np.where(keep, s, -np.inf)
+    mx = s.max(-1, keepdims=True)
+    w = np.exp(s - mx)
+    return np.einsum("bhik,bhkd->bhid", w, v) / w.sum(-1, keepdims=True)
+
+
+def brute_decisions(s, Br, Bc, tau):
+    """Skip decisions from the definition: the running max before tile j is the
+    max of all visible scores in tiles < j (skipped tiles never exceed it)."""
+    B, H, N, _ = s.shape
+    n_rb, n_t = -(-N // Br), -(-N // Bc)
+    mask = np.full((B, H, n_rb, n_t), 2, np.uint8)
+    margin = np.full((B, H, n_rb, n_t), np.nan)
+    for b in range(B):
+        for h in range(H):
+            for rb in range(n_rb):
+                r0, r1 = rb * Br, min(N, rb * Br + Br)
+                for j in range(n_t):
+                    c0, c1 = j * Bc, min(N, j * Bc + Bc)
+                    if np.all(np.isneginf(s[b, h, r0:r1, c0:c1])) and c0 > r1 - 1:
+                        continue                               # never visited (causal)
+                    rows = []
+                    for r in range(r0, r1):
+                        prev = s[b, h, r, :c0]
+                        m = prev.max() if prev.size else -np.inf
+                        mt = s[b, h, r, c0:c1].max()
+                        if m == -np.inf:
+                            rows.append(np.inf)
+                        elif mt == -np.inf:
+                            rows.append(-np.inf)
+                        else:
+                            rows.append(mt - m + tau)
+                    mg = max(rows)
+                    margin[b, h, rb, j] = mg
+                    mask[b, h, rb, j] = 1 if mg < 0 else 0
+    return mask, margin
+
+
+def kept_keys(mask, N, Br, Bc):
+    """Boolean [B,H,N,N]: key k is used by row i (its tile was kept for i's row block)."""
+    B, H, n_rb, n_t = mask.shape
+    keep = np.zeros((B, H, N, N), bool)
+    for rb in range(n_rb):
+        for j in range(n_t):
+            sel = mask[:, :, rb, j] == 0
+            keep[:, :, rb * Br:(rb + 1) * Br, j * Bc:(j + 1) * Bc] |= sel[:, :, None, None]
+    return keep
+
+
+def skippy(B=1, Hq=2, Hkv=1, N=200, d=64, seed=3, q_u=8.0, sink=6.0, q_sigma=2.0):
+    """Inputs on which many tiles skip: a strong shared direction u in every
+    query and a few sink keys along u."""
+    return inputs.prefill_inputs(B, Hq, Hkv, N, d, seed=seed, q_sigma=q_sigma, q_u=q_u,
+                                 sink_scale=sink, n_sinks=4)
+
+
+SHAPES = [  # B, Hq, Hkv, N, d, causal, Br, Bc
+    (1, 1, 1, 1, 64, True, 64, 64),
+    (1, 1, 1, 7, 64, False, 64, 64),
+    (1, 2, 2, 64, 64, True, 64, 64),
+    (2, 2, 1, 65, 64, True, 64, 64),
+    (1, 4, 2, 200, 128, True, 128, 64),
+    (1, 2, 1, 256, 128, False, 128, 128),
+    (1, 1, 1, 200, 64, True, 64, 128),
+]
+
+
+# ----------------------------------------------------------------------------
+# pins
+# ----------------------------------------------------------------------------
+
+@pin
+def pin_exact_equals_bruteforce(lib):
+    """tau = inf is exact softmax(QK^T/sqrt d)V: brute force on tiny inputs."""
+    for i, (B, Hq, Hkv, N, d, causal, Br, Bc) in enumerate(SHAPES):
+        Q, K, V = inputs.prefill_inputs(B, Hq, Hkv, N, d, seed=10 + i, q_sigma=1.5)
+        ref = softmax_av(scores(Q, K, causal), V)
+        r = oracle.prefill(Q, K, V, causal, math.inf, Br, Bc, lib_path=lib)
+        np.testing.assert_allclose(r["O"], ref, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(r["O_exact"], ref, rtol=0, atol=1e-12)
+        assert np.all(r["mask"][r["mask"] != 2] == 0)
+
+
+@pin
+def pin_uniform_logits_give_mean_of_v(lib):
+    """Q = 0 makes every logit equal: O is the mean of the visible V rows
+    (the prefix mean under causal attention)."""
+    for causal in (False, True):
+        _, K, V = inputs.prefill_inputs(1, 2, 1, 130, 64, seed=4)
+        Q = torch.zeros(1, 2, 130, 64, dtype=torch.bfloat16)
+        r = oracle.prefill(Q, K, V, causal, 3.0, 64, 64, lib_path=lib)
+        v = f64(V)[0, 0]
+        if causal:
+            mean = np.cumsum(v, 0) / np.arange(1, 131)[:, None]
+        else:
+            mean = np.broadcast_to(v.mean(0), v.shape)
+        for h in range(2):
+            np.testing.assert_allclose(r["O"][0, h], mean, rtol=0, atol=1e-12)
+
+
+@pin
+def pin_one_logit_closed_form(lib):
+    """Logits {a at key j*, 0 elsewhere}: O = (e^a V[j*] + sum_{k!=j*} V[k]) / (e^a + N - 1).
+    Pins the exponential base and the 1/sqrt(d) scale."""
+    N, d = 96, 64
+    _, _, V = inputs.prefill_inputs(1, 1, 1, N, d, seed=5)
+    Q = torch.zeros(1, 1, N, d, dtype=torch.bfloat16)
+    Q[..., 0] = 8.0                                     # q . k / sqrt(64) = K[k, 0]
+    K = torch.zeros(1, 1, N, d, dtype=torch.bfloat16)
+    for a, js in ((3.0, 70), (40.0, 17)):
+        K.zero_()
+        K[0, 0, js, 0] = a
+        v = f64(V)[0, 0]
+        expect = (math.exp(a) * v[js] + v.sum(0) - v[js]) / (math.exp(a) + N - 1)
+        r = oracle.prefill(Q, K, V, False, math.inf, 64, 64, lib_path=lib)
+        np.testing.assert_allclose(r["O"][0, 0], np.broadcast_to(expect, (N, d)), rtol=1e-13, atol=1e-14)
+        if a == 40.0:                                   # one dominant logit -> that V row
+            bound = 2 * np.abs(v).max() * (N - 1) * math.exp(-a)
+            assert np.abs(r["O"][0, 0] - v[js]).max() <= bound
+
+
+@pin
+def pin_rows_sum_to_one(lib):
+    """With V = 1 every output is the row sum of the (kept) probabilities: 1."""
+    Q, K, _ = skippy(N=200)
+    V = torch.ones(1, 1, 200, 64, dtype=torch.bfloat16)
+    for tau in (0.0, 2.0, 8.0, math.inf):
+        for causal in (False, True):
+            r = oracle.prefill(Q, K, V, causal, tau, 64, 64, lib_path=lib)
+            np.testing.assert_allclose(r["O"], 1.0, rtol=0, atol=1e-13)
+
+
+@pin
+def pin_skip_error_bound(lib):
+    """|O_skip - O_exact| <= 2 max|V| p_r, with p_r the skipped softmax mass."""
+    Q, K, V = skippy(N=256)
+    vmax = np.abs(f64(V)).max()
+    saw_skip = False
+    for tau in (0.5, 4.0, 16.0):
+        for causal in (False, True):
+            r = oracle.prefill(Q, K, V, causal, tau, 64, 64, lib_path=lib)
+            saw_skip |= bool((r["mask"] == 1).any())
+            dev = np.abs(r["O"] - r["O_exact"]).max(-1)
+            assert np.all(dev <= 2 * vmax * r["pskip"] + 1e-12)
+            # the skipped mass is exactly the mass of the keys in skipped tiles
+            s = scores(Q, K, causal)
+            w = np.exp(s - s.max(-1, keepdims=True))
+            skipped = ~kept_keys(r["mask"], 256, 64, 64) & np.isfinite(s)
+            np.testing.assert_allclose(r["pskip"], (w * skipped).sum(-1) / w.sum(-1), rtol=0, atol=1e-12)
+    assert saw_skip
+
+
+@pin
+def pin_output_is_softmax_over_kept_tiles(lib):
+    """Given the skip set, O is plain softmax restricted to the kept tiles (two-pass form)."""
+    for (Br, Bc) in ((64, 64), (128, 64), (64, 128)):
+        Q, K, V = skippy(N=200, Hq=2, Hkv=1)
+        for causal in (False, True):
+            r = oracle.prefill(Q, K, V, causal, 3.0, Br, Bc, lib_path=lib)
+            keep = kept_keys(r["mask"], 200, Br, Bc)
+            ref = softmax_av(scores(Q, K, causal), V, keep)
+            np.testing.assert_allclose(r["O"], ref, rtol=0, atol=1e-12)
+
+
+@pin
+def pin_decisions_from_prefix_max(lib):
+    """Mask and margin equal those derived from the exact prefix row max."""
+    for (Br, Bc, N) in ((64, 64, 200), (128, 64, 256), (64, 128, 190)):
+        Q, K, V = skippy(N=N, Hq=2, Hkv=1, seed=Br + Bc + N)
+        for causal in (False, True):
+            s = scores(Q, K, causal)
+            for tau in (0.0, 1.5, 6.0):
+                r = oracle.prefill(Q, K, V, causal, tau, Br, Bc, lib_path=lib)
+                mask, margin = brute_decisions(s, Br, Bc, tau)
+                np.testing.assert_array_equal(r["mask"], mask)
+                np.testing.assert_allclose(r["margin"], margin, rtol=0, atol=1e-10)
+
+
+def read_golden():
+    rows = []
+    for line in open(GOLDEN):
+        line = line.split("#")[0].strip()
+        if line:
+            t, m0, m1, mg = line.split()
+            rows.append((float(t), int(m0), int(m1), float(mg)))
+    return rows
+
+
+@pin
+def pin_golden_two_tile_example(lib):
+    """The hand-built example: tile 1 is skipped iff tau < 5 (strict)."""
+    N, d = 128, 64
+    Q = torch.zeros(1, 1, N, d, dtype=torch.bfloat16)
+    Q[..., 0] = 8.0
+    K = torch.zeros(1, 1, N, d, dtype=torch.bfloat16)
+    K[0, 0, 0, 0], K[0, 0, 64, 0] = 10.0, 5.0
+    V = torch.zeros(1, 1, N, d, dtype=torch.bfloat16)
+    V[0, 0, 0, 0], V[0, 0, 64, 1], V[0, 0, :, 2] = 1.0, 1.0, 1.0
+    z_skip, z_keep = math.exp(10) + 63, math.exp(10) + 63 + math.exp(5) + 63
+    rows = read_golden()
+    assert len(rows) == 5
+    for tau, m0, m1, mg in rows:
+        r = oracle.prefill(Q, K, V, False, tau, 64, 64, lib_path=lib)
+        for rb in range(2):
+            assert r["mask"][0, 0, rb, 0] == m0 and r["mask"][0, 0, rb, 1] == m1
+            assert r["margin"][0, 0, rb, 0] == math.inf
+            if math.isinf(mg):
+                assert r["margin"][0, 0, rb, 1] == math.inf
+            else:
+                assert abs(r["margin"][0, 0, rb, 1] - mg) < 1e-12
+        o = r["O"][0, 0]
+        if m1:
+            expect = (math.exp(10) / z_skip, 0.0, 1.0)
+            np.testing.assert_allclose(r["pskip"][0, 0], (math.exp(5) + 63) / z_keep, rtol=1e-13)
+        else:
+            expect = (math.exp(10) / z_keep, math.exp(5) / z_keep, 1.0)
+            np.testing.assert_allclose(r["pskip"][0, 0], 0.0, atol=0)
+        for c in range(3):
+            np.testing.assert_allclose(o[:, c], expect[c], rtol=1e-13, atol=1e-15)
+        np.testing.assert_allclose(o[:, 3:], 0.0, atol=0)
+
+
+@pin
+def pin_tau_monotone_and_limits(lib):
+    """Skip sets shrink as tau grows; tile 0 is never skipped; tau=inf skips nothing."""
+    Q, K, V = skippy(N=256, Hq=2, Hkv=2)
+    prev = None
+    for tau in (0.0, 0.5, 2.0, 8.0, 32.0, math.inf):
+        r = oracle.prefill(Q, K, V, True, tau, 64, 64, lib_path=lib)
+        sk = r["mask"] == 1
+        assert not sk[..., 0].any()
+        if prev is not None:
+            assert np.all(sk <= prev)           # skipped at larger tau => skipped at smaller
+        prev = sk
+    assert not prev.any()
+
+
+@pin
+def pin_gqa_equals_repeated_heads(lib):
+    """Hkv < Hq gives the same result as Hkv = Hq with each KV head repeated g times."""
+    Q, K, V = skippy(N=130, Hq=4, Hkv=2, seed=7)
+    Kr, Vr = K.repeat_interleave(2, dim=1), V.repeat_interleave(2, dim=1)
+    for tau in (1.0, math.inf):
+        a = oracle.prefill(Q, K, V, True, tau, 64, 64, lib_path=lib)
+        b = oracle.prefill(Q, Kr, Vr, True, tau, 64, 64, lib_path=lib)
+        np.testing.assert_array_equal(a["O"], b["O"])
+        np.testing.assert_array_equal(a["mask"], b["mask"])
+
+
+@pin
+def pin_causal_first_row_is_v0(lib):
+    """Under causal attention query 0 sees only key 0: O[0] = V[0] exactly."""
+    Q, K, V = inputs.prefill_inputs(1, 2, 2, 70, 64, seed=8)
+    r = oracle.prefill(Q, K, V, True, 1.0, 64, 64, lib_path=lib)
+    np.testing.assert_array_equal(r["O"][0, :, 0], f64(V)[0, :, 0])
+
+
+@pin
+def pin_row_block_subset_is_exact(lib):
+    """Computing a subset of row blocks gives bit-identical results for them."""
+    Q, K, V = skippy(N=256, Hq=2, Hkv=1, seed=9)
+    full = oracle.prefill(Q, K, V, True, 2.0, 64, 64, lib_path=lib)
+    units = [(0, 1, 3), (0, 0, 0), (0, 1, 1)]
+    sub = oracle.prefill(Q, K, V, True, 2.0, 64, 64, units=units, lib_path=lib)
+    for b, h, rb in units:
+        np.testing.assert_array_equal(sub["O"][b, h, rb * 64:(rb + 1) * 64], full["O"][b, h, rb * 64:(rb + 1) * 64])
+        np.testing.assert_array_equal(sub["mask"][b, h, rb], full["mask"][b, h, rb])
+    assert np.isnan(sub["O"][0, 0, 64:128]).all()
+
+
+# ---------------------------------------------------------------- decode pins
+
+def dec_inputs(B=2, Hq=4, Hkv=2, L=300, d=64, seed=11, q_u=8.0, sink=6.0):
+    return inputs.decode_inputs(B, Hq, Hkv, L, d, seed=seed, q_sigma=2.0, q_u=q_u,
+                                sink_scale=sink, n_sinks=4)
+
+
+def dec_scores(q, K):
+    qq, k = f64(q), f64(K)
+    g = qq.shape[1] // k.shape[1]
+    k = np.repeat(k, g, axis=1)
+    return np.einsum("bhd,bhkd->bhk", qq, k) / math.sqrt(qq.shape[-1])
+
+
+@pin
+def pin_decode_exact_equals_bruteforce(lib):
+    q, K, V = dec_inputs()
+    s = dec_scores(q, K)
+    v = np.repeat(f64(V), 2, axis=1)
+    w = np.exp(s - s.max(-1, keepdims=True))
+    ref = np.einsum("bhk,bhkd->bhd", w, v) / w.sum(-1, keepdims=True)
+    for Ls in (64, 128, 320):                    # split layout does not change exact results
+        r = oracle.decode(q, K, V, math.inf, Ls, 64, lib_path=lib)
+        np.testing.assert_allclose(r["o"], ref, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(r["o_exact"], ref, rtol=0, atol=1e-12)
+        assert not (r["mask"] == 1).any()
+
+
+@pin
+def pin_decode_decisions_split_local(lib):
+    """Decode rows are the g heads of a KV group; the running max restarts at
+    each split; output = softmax over kept tiles; bound holds; V=1 gives 1."""
+    q, K, V = dec_inputs(L=640)
+    s = dec_scores(q, K)                          # [B,Hq,L]
+    B, Hq, L = s.shape
+    g, Bt = 2, 64
+    saw = False
+    for Ls in (128, 320, 640):
+        for tau in (0.0, 2.0, 6.0):
+            r = oracle.decode(q, K, V, tau, Ls, Bt, lib_path=lib)
+            keep = np.zeros_like(s, bool)
+            for b in range(B):
+                for kv in range(Hq // g):
+                    rows = s[b, kv * g:(kv + 1) * g]
+                    for j in range(-(-L // Bt)):
+                        c0, c1 = j * Bt, min(L, j * Bt + Bt)
+                        split0 = (c0 // Ls) * Ls
+                        m = rows[:, split0:c0].max(-1) if c0 > split0 else np.full(g, -np.inf)
+                        mt = rows[:, c0:c1].max(-1)
+                        mg = max(np.inf if mm == -np.inf else t - mm + tau for t, mm in zip(mt, m))
+                        assert r["mask"][b, kv, j] == (1 if mg < 0 else 0)
+                        if np.isfinite(mg):
+                            assert abs(r["margin"][b, kv, j] - mg) < 1e-10
+                        if mg >= 0:
+                            keep[b, kv * g:(kv + 1) * g, c0:c1] = True
+            saw |= bool((r["mask"] == 1).any())
+            w = np.where(keep, np.exp(s - s.max(-1, keepdims=True)), 0.0)
+            v = np.repeat(f64(V), g, axis=1)
+            ref = np.einsum("bhk,bhkd->bhd", w, v) / w.sum(-1, keepdims=True)
+            np.testing.assert_allclose(r["o"], ref, rtol=0, atol=1e-12)
+            dev = np.abs(r["o"] - r["o_exact"]).max(-1)
+            assert np.all(dev <= 2 * np.abs(f64(V)).max() * r["pskip"] + 1e-12)
+    assert saw
+    ones = torch.ones_like(V)
+    np.testing.assert_allclose(oracle.decode(q, K, ones, 1.0, 128, 64, lib_path=lib)["o"], 1.0, atol=1e-13)
+
+
+@pin
+def pin_decode_matches_prefill_single_row(lib):
+    """g = 1 and one split: decode of q equals prefill row 0 of a non-causal
+    problem whose first query is q, with one-row row blocks and 64-key tiles."""
+    q, K, V = dec_inputs(B=1, Hq=1, Hkv=1, L=256, seed=12)
+    Q = torch.zeros(1, 1, 256, 64, dtype=torch.bfloat16)
+    Q[0, 0, 0] = q[0, 0]
+    for tau in (0.0, 3.0, math.inf):
+        d_ = oracle.decode(q, K, V, tau, 256, 64, lib_path=lib)
+        p_ = oracle.prefill(Q, K, V, False, tau, 1, 64, units=[(0, 0, 0)], lib_path=lib)
+        np.testing.assert_allclose(d_["o"][0, 0], p_["O"][0, 0, 0], rtol=0, atol=1e-13)
+        np.testing.assert_array_equal(d_["mask"][0, 0], p_["mask"][0, 0, 0])
+
+
+@pytest.mark.parametrize("fn", PINS, ids=[f.__name__ for f in PINS])
+def test_pin(fn):
+    fn(None)
