@@ -1,0 +1,189 @@
+"""Skip Softmax attention for NVIDIA B200 (sm_100a): Python binding of libattn.so.
+
+The functions named like the C ABI (``attn_prefill``, ``attn_decode`` ...)
+take raw device pointers and sizes and only marshal arguments; the torch
+helpers ``prefill`` and ``decode`` take tensors and pass their pointers.
+Every step of the computation runs in the library's CUDA kernels.  There is
+no CPU fallback: if the library cannot be loaded, or no sm_100 device is
+present, calls raise ``AttnError``.
+
+Method: "Accelerating Long-Context Inference with Skip Softmax in NVIDIA
+TensorRT-LLM" (Key Points; Detailed Analysis) -- a key tile is skipped when
+every query row's tile maximum is below its running maximum minus tau.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+__all__ = [
+    "AttnError", "lib", "attn_prefill", "attn_prefill_ex", "attn_decode", "attn_decode_ex",
+    "attn_decode_split_len", "attn_decode_tile", "attn_decode_workspace_bytes",
+    "attn_set_stream", "attn_sync_status", "attn_last_timeout_site", "attn_set_wait_limit_ms",
+    "attn_status_string", "attn_shutdown", "prefill", "decode", "STATUS",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libattn.so")
+STATUS = {0: "ATTN_OK", 1: "ATTN_ERR_INVALID_ARG", 2: "ATTN_ERR_UNSUPPORTED", 3: "ATTN_ERR_CUDA",
+          4: "ATTN_ERR_TIMEOUT"}
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__(f"{what} failed: {STATUS.get(status, status)}")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load libattn.so (built in-tree by ``block_skipping_softmax_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise AttnError(-1, f"loading {LIB_PATH} (not built; run python -m block_skipping_softmax_b200.build)")
+    L = ctypes.CDLL(LIB_PATH)
+    vp, ci, cf, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    sig = {
+        "attn_prefill": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, ci]),
+        "attn_prefill_ex": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, ci, vp, vp]),
+        "attn_decode": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf]),
+        "attn_decode_ex": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, vp, vp, vp, sz]),
+        "attn_decode_split_len": (ci, [ci, ci, ci]),
+        "attn_decode_tile": (ci, []),
+        "attn_decode_workspace_bytes": (sz, [ci, ci, ci, ci, ci]),
+        "attn_set_stream": (ci, [vp]),
+        "attn_sync_status": (ci, []),
+        "attn_last_timeout_site": (ci, []),
+        "attn_set_wait_limit_ms": (ci, [ci]),
+        "attn_status_string": (ctypes.c_char_p, [ci]),
+        "attn_shutdown": (None, []),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(L, name)
+        f.restype, f.argtypes = res, args
+    _lib = L
+    return L
+
+
+# ---- C-ABI names: argument marshalling only ---------------------------------
+
+def attn_prefill(Q, K, V, O, B, Hq, Hkv, N, d, causal, tau, Br, Bc) -> int:
+    return lib().attn_prefill(Q, K, V, O, B, Hq, Hkv, N, d, int(causal), float(tau), Br, Bc)
+
+
+def attn_prefill_ex(Q, K, V, O, B, Hq, Hkv, N, d, causal, tau, Br, Bc, stream=None, skip_mask=None) -> int:
+    return lib().attn_prefill_ex(Q, K, V, O, B, Hq, Hkv, N, d, int(causal), float(tau), Br, Bc,
+                                 stream, skip_mask)
+
+
+def attn_decode(q, K, V, o, B, Hq, Hkv, L, d, tau) -> int:
+    return lib().attn_decode(q, K, V, o, B, Hq, Hkv, L, d, float(tau))
+
+
+def attn_decode_ex(q, K, V, o, B, Hq, Hkv, L, d, tau, stream=None, skip_mask=None, ws=None, ws_bytes=0) -> int:
+    return lib().attn_decode_ex(q, K, V, o, B, Hq, Hkv, L, d, float(tau), stream, skip_mask, ws, ws_bytes)
+
+
+def attn_decode_split_len(B, Hkv, L) -> int:
+    return lib().attn_decode_split_len(B, Hkv, L)
+
+
+def attn_decode_tile() -> int:
+    return lib().attn_decode_tile()
+
+
+def attn_decode_workspace_bytes(B, Hq, Hkv, L, d) -> int:
+    return lib().attn_decode_workspace_bytes(B, Hq, Hkv, L, d)
+
+
+def attn_set_stream(stream) -> int:
+    return lib().attn_set_stream(stream)
+
+
+def attn_sync_status() -> int:
+    return lib().attn_sync_status()
+
+
+def attn_last_timeout_site() -> int:
+    return lib().attn_last_timeout_site()
+
+
+def attn_set_wait_limit_ms(ms) -> int:
+    return lib().attn_set_wait_limit_ms(int(ms))
+
+
+def attn_status_string(status) -> str:
+    return lib().attn_status_string(int(status)).decode()
+
+
+def attn_shutdown() -> None:
+    lib().attn_shutdown()
+
+
+# ---- torch helpers: pass tensor pointers, no compute -------------------------
+
+def _check(st: int, what: str):
+    if st != 0:
+        raise AttnError(st, what)
+
+
+def _stream_ptr(stream):
+    import torch
+
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return s.cuda_stream
+
+
+def prefill(Q, K, V, causal: bool, tau: float = math.inf, Br: int = 128, Bc: int = 128,
+            out=None, skip_mask: bool = False, stream=None):
+    """O = Skip Softmax attention of bf16 CUDA tensors Q [B,Hq,N,d], K/V [B,Hkv,N,d].
+
+    Returns O (and the uint8 skip mask [B,Hq,ceil(N/Br),ceil(N/Bc)] when asked).
+    """
+    import torch
+
+    B, Hq, N, d = Q.shape
+    Hkv = K.shape[1]
+    for t in (Q, K, V):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise AttnError(1, "prefill (tensors must be contiguous bf16 CUDA tensors)")
+    O = out if out is not None else torch.empty_like(Q)
+    mask = None
+    if skip_mask:
+        mask = torch.empty(B, Hq, -(-N // Br), -(-N // Bc), dtype=torch.uint8, device=Q.device)
+    st = attn_prefill_ex(Q.data_ptr(), K.data_ptr(), V.data_ptr(), O.data_ptr(), B, Hq, Hkv, N, d,
+                         causal, tau, Br, Bc, _stream_ptr(stream),
+                         mask.data_ptr() if mask is not None else None)
+    _check(st, "attn_prefill_ex")
+    return (O, mask) if skip_mask else O
+
+
+def decode(q, K, V, tau: float = math.inf, out=None, skip_mask: bool = False, stream=None,
+           workspace=None):
+    """o = Skip Softmax decode attention: q [B,Hq,d], K/V [B,Hkv,L,d] bf16 CUDA tensors.
+
+    ``workspace``: optional uint8 CUDA tensor of at least
+    attn_decode_workspace_bytes(...) bytes; otherwise the library's own is used.
+    """
+    import torch
+
+    B, Hq, d = q.shape
+    Hkv, L = K.shape[1], K.shape[2]
+    for t in (q, K, V):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise AttnError(1, "decode (tensors must be contiguous bf16 CUDA tensors)")
+    o = out if out is not None else torch.empty_like(q)
+    mask = None
+    if skip_mask:
+        mask = torch.empty(B, Hkv, -(-L // attn_decode_tile()), dtype=torch.uint8, device=q.device)
+    ws, wsb = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel())
+    st = attn_decode_ex(q.data_ptr(), K.data_ptr(), V.data_ptr(), o.data_ptr(), B, Hq, Hkv, L, d,
+                        tau, _stream_ptr(stream), mask.data_ptr() if mask is not None else None,
+                        ws, wsb)
+    _check(st, "attn_decode_ex")
+    return (o, mask) if skip_mask else o

@@ -1,0 +1,289 @@
+// C ABI of libattn.so: argument validation, device checks, workspace and the
+// device status word.  Every compute step runs in the kernels; this layer only
+// checks arguments, encodes TMA descriptors (in the launchers) and launches.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "attn.h"
+#include "kernels.cuh"
+
+namespace {
+
+__device__ int g_status;  // 0, or ATTN_DEVICE_TIMEOUT_BASE + site of a wait that gave up
+
+constexpr int kMaxDevices = 64;
+constexpr float kLog2e = 1.4426950408889634f;
+
+std::mutex g_mu;
+cudaStream_t g_stream = nullptr;
+unsigned long long g_wait_limit_ns = 2000ull * 1000ull * 1000ull;
+int g_last_site = 0;
+int g_dev_checked[kMaxDevices];  // 0 unknown, 1 sm_100, 2 other
+int* g_status_ptr[kMaxDevices];
+void* g_ws[kMaxDevices];
+size_t g_ws_bytes[kMaxDevices];
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Device check and per-device status word; returns ATTN_OK or an error.
+int device_ready(int* dev_out, int** status_out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_UNSUPPORTED;
+  if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_dev_checked[dev] == 0) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return ATTN_ERR_CUDA;
+    g_dev_checked[dev] = (prop.major == 10 && prop.minor == 0) ? 1 : 2;
+    if (g_dev_checked[dev] == 1) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) {
+        g_dev_checked[dev] = 0;
+        return ATTN_ERR_CUDA;
+      }
+      g_status_ptr[dev] = static_cast<int*>(p);
+    }
+  }
+  if (g_dev_checked[dev] != 1) return ATTN_ERR_UNSUPPORTED;
+  *dev_out = dev;
+  *status_out = g_status_ptr[dev];
+  return ATTN_OK;
+}
+
+bool tau_ok(float tau) { return !std::isnan(tau) && tau >= 0.f; }
+
+int check_prefill(const void* Q, const void* K, const void* V, const void* O, int B, int Hq,
+                  int Hkv, int N, int d, float tau, int Br, int Bc) {
+  if (!Q || !K || !V || !O) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return ATTN_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || N <= 0) return ATTN_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_INVALID_ARG;
+  if (!((Br == 64 && Bc == 64) || (Br == 128 && Bc == 64) || (Br == 128 && Bc == 128)))
+    return ATTN_ERR_INVALID_ARG;
+  if (!tau_ok(tau)) return ATTN_ERR_INVALID_ARG;
+  const long long n_rb = (N + Br - 1) / Br;
+  if (n_rb * B * Hq > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  return ATTN_OK;
+}
+
+int check_decode(const void* q, const void* K, const void* V, const void* o, int B, int Hq,
+                 int Hkv, int L, int d, float tau) {
+  if (!q || !K || !V || !o) return ATTN_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(o)) return ATTN_ERR_INVALID_ARG;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || L <= 0) return ATTN_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return ATTN_ERR_INVALID_ARG;
+  if (!tau_ok(tau)) return ATTN_ERR_INVALID_ARG;
+  const int g = Hq / Hkv;
+  if (g != 1 && g != 2 && g != 4 && g != 8) return ATTN_ERR_UNSUPPORTED;
+  if (Hkv > 65535 || B > 65535) return ATTN_ERR_UNSUPPORTED;
+  return ATTN_OK;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+void decode_ws_layout(int B, int Hq, int n_splits, int d, size_t* o_bytes, size_t* total) {
+  *o_bytes = align256(static_cast<size_t>(B) * Hq * n_splits * d * sizeof(float));
+  *total = *o_bytes + align256(static_cast<size_t>(B) * Hq * n_splits * sizeof(float));
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_prefill_ex(const void* Q, const void* K, const void* V, void* O, int B, int Hq, int Hkv,
+                    int N, int d, int causal, float tau, int Br, int Bc, void* stream,
+                    uint8_t* skip_mask) {
+  int st = check_prefill(Q, K, V, O, B, Hq, Hkv, N, d, tau, Br, Bc);
+  if (st != ATTN_OK) return st;
+  int dev = 0;
+  int* status = nullptr;
+  if ((st = device_ready(&dev, &status)) != ATTN_OK) return st;
+  bss::PrefillLaunch a{};
+  a.Q = Q;
+  a.K = K;
+  a.V = V;
+  a.O = O;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.N = N;
+  a.d = d;
+  a.causal = causal ? 1 : 0;
+  a.Br = Br;
+  a.Bc = Bc;
+  a.scale_log2 = kLog2e / std::sqrt(static_cast<float>(d));
+  a.tau_is_inf = std::isinf(tau) ? 1 : 0;
+  a.tau_log2 = a.tau_is_inf ? 0.f : tau * kLog2e;
+  a.skip_mask = skip_mask;
+  a.status = status;
+  a.wait_limit_ns = g_wait_limit_ns;
+  a.stream = static_cast<cudaStream_t>(stream);
+  return bss::launch_prefill(a);
+}
+
+int attn_prefill(const void* Q, const void* K, const void* V, void* O, int B, int Hq, int Hkv,
+                 int N, int d, int causal, float tau, int Br, int Bc) {
+  return attn_prefill_ex(Q, K, V, O, B, Hq, Hkv, N, d, causal, tau, Br, Bc, g_stream, nullptr);
+}
+
+int attn_decode_tile(void) { return bss::kDecodeTile; }
+
+int attn_decode_split_len(int B, int Hkv, int L) {
+  if (B <= 0 || Hkv <= 0 || L <= 0) return -1;
+  // Choose tiles-per-split to minimise modelled time: waves of 296 resident
+  // CTAs (148 SMs x 2) times (tiles per CTA + ~2 tiles of start-up cost).
+  const long long slots = 296;
+  const long long groups = static_cast<long long>(B) * Hkv;
+  const long long n_tiles = (L + bss::kDecodeTile - 1) / bss::kDecodeTile;
+  long long best_tps = n_tiles, best_cost = -1;
+  for (long long tps = n_tiles; tps >= 1; --tps) {
+    const long long ns = (n_tiles + tps - 1) / tps;
+    if (ns > 4096) break;
+    const long long waves = (groups * ns + slots - 1) / slots;
+    const long long cost = waves * (tps + 2);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best_tps = tps;
+    }
+  }
+  return static_cast<int>(best_tps * bss::kDecodeTile);
+}
+
+size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int L, int d) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || L <= 0 || (d != 64 && d != 128)) return 0;
+  const int ls = attn_decode_split_len(B, Hkv, L);
+  const int n_splits = (L + ls - 1) / ls;
+  size_t ob = 0, total = 0;
+  decode_ws_layout(B, Hq, n_splits, d, &ob, &total);
+  return total;
+}
+
+int attn_decode_ex(const void* q, const void* K, const void* V, void* o, int B, int Hq, int Hkv,
+                   int L, int d, float tau, void* stream, uint8_t* skip_mask, void* ws,
+                   size_t ws_bytes) {
+  int st = check_decode(q, K, V, o, B, Hq, Hkv, L, d, tau);
+  if (st != ATTN_OK) return st;
+  if (ws == nullptr && ws_bytes != 0) return ATTN_ERR_INVALID_ARG;
+  if (ws != nullptr && (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return ATTN_ERR_INVALID_ARG;
+  int dev = 0;
+  int* status = nullptr;
+  if ((st = device_ready(&dev, &status)) != ATTN_OK) return st;
+  const int ls = attn_decode_split_len(B, Hkv, L);
+  const int n_splits = (L + ls - 1) / ls;
+  size_t ob = 0, need = 0;
+  decode_ws_layout(B, Hq, n_splits, d, &ob, &need);
+  if (ws == nullptr) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_ws_bytes[dev] < need) {
+      // the old buffer may still be read by queued work on another stream
+      if (g_ws[dev]) {
+        cudaDeviceSynchronize();
+        cudaFree(g_ws[dev]);
+        g_ws[dev] = nullptr;
+        g_ws_bytes[dev] = 0;
+      }
+      if (cudaMalloc(&g_ws[dev], need) != cudaSuccess) return ATTN_ERR_CUDA;
+      g_ws_bytes[dev] = need;
+    }
+    ws = g_ws[dev];
+  } else if (ws_bytes < need) {
+    return ATTN_ERR_INVALID_ARG;
+  }
+  bss::DecodeLaunch a{};
+  a.q = q;
+  a.K = K;
+  a.V = V;
+  a.o = o;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.L = L;
+  a.d = d;
+  a.scale_log2 = kLog2e / std::sqrt(static_cast<float>(d));
+  a.tau_is_inf = std::isinf(tau) ? 1 : 0;
+  a.tau_log2 = a.tau_is_inf ? 0.f : tau * kLog2e;
+  a.split_len = ls;
+  a.n_splits = n_splits;
+  a.o_part = static_cast<float*>(ws);
+  a.lse_part = reinterpret_cast<float*>(static_cast<char*>(ws) + ob);
+  a.skip_mask = skip_mask;
+  a.status = status;
+  a.wait_limit_ns = g_wait_limit_ns;
+  a.stream = static_cast<cudaStream_t>(stream);
+  return bss::launch_decode(a);
+}
+
+int attn_decode(const void* q, const void* K, const void* V, void* o, int B, int Hq, int Hkv,
+                int L, int d, float tau) {
+  return attn_decode_ex(q, K, V, o, B, Hq, Hkv, L, d, tau, g_stream, nullptr, nullptr, 0);
+}
+
+int attn_set_stream(void* stream) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_stream = static_cast<cudaStream_t>(stream);
+  return ATTN_OK;
+}
+
+int attn_set_wait_limit_ms(int ms) {
+  if (ms < 1) return ATTN_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_wait_limit_ns = static_cast<unsigned long long>(ms) * 1000000ull;
+  return ATTN_OK;
+}
+
+int attn_sync_status(void) {
+  int dev = 0;
+  int* status = nullptr;
+  int st = device_ready(&dev, &status);
+  if (st != ATTN_OK) return st;
+  if (cudaDeviceSynchronize() != cudaSuccess) return ATTN_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return ATTN_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    g_last_site = v - ATTN_DEVICE_TIMEOUT_BASE;
+    return ATTN_ERR_TIMEOUT;
+  }
+  return ATTN_OK;
+}
+
+int attn_last_timeout_site(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  return g_last_site;
+}
+
+const char* attn_status_string(int s) {
+  switch (s) {
+    case ATTN_OK: return "ATTN_OK";
+    case ATTN_ERR_INVALID_ARG: return "ATTN_ERR_INVALID_ARG";
+    case ATTN_ERR_UNSUPPORTED: return "ATTN_ERR_UNSUPPORTED";
+    case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA";
+    case ATTN_ERR_TIMEOUT: return "ATTN_ERR_TIMEOUT";
+    default: return "ATTN_ERR_UNKNOWN";
+  }
+}
+
+void attn_shutdown(void) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  int cur = 0;
+  const bool have = cudaGetDevice(&cur) == cudaSuccess;
+  for (int dev = 0; dev < kMaxDevices; ++dev) {
+    if (!g_ws[dev]) continue;
+    if (cudaSetDevice(dev) == cudaSuccess) {
+      cudaDeviceSynchronize();
+      cudaFree(g_ws[dev]);
+    }
+    g_ws[dev] = nullptr;
+    g_ws_bytes[dev] = 0;
+  }
+  if (have) cudaSetDevice(cur);
+}
+
+}  // extern "C"

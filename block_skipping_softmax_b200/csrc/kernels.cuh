@@ -1,0 +1,53 @@
+// Internal launch descriptors shared by the C-ABI layer and the kernels.
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+
+#include <cstddef>
+#include <cstdint>
+
+#include "attn.h"
+
+namespace bss {
+
+struct PrefillLaunch {
+  const void* Q;
+  const void* K;
+  const void* V;
+  void* O;
+  int B, Hq, Hkv, N, d, causal, Br, Bc;
+  float scale_log2;  // log2(e) / sqrt(d): scores in log2 units
+  float tau_log2;    // tau * log2(e)
+  int tau_is_inf;
+  uint8_t* skip_mask;
+  int* status;
+  unsigned long long wait_limit_ns;
+  cudaStream_t stream;
+};
+
+int launch_prefill(const PrefillLaunch& a);
+
+constexpr int kDecodeTile = 64;  // keys per decode tile
+
+struct DecodeLaunch {
+  const void* q;
+  const void* K;
+  const void* V;
+  void* o;
+  int B, Hq, Hkv, L, d;
+  float scale_log2;
+  float tau_log2;
+  int tau_is_inf;
+  int split_len;  // keys per split, multiple of kDecodeTile
+  int n_splits;
+  float* o_part;    // [B*Hq, n_splits, d] fp32 (normalised partial outputs)
+  float* lse_part;  // [B*Hq, n_splits]    fp32 (log2-sum-exp of each split)
+  uint8_t* skip_mask;
+  int* status;
+  unsigned long long wait_limit_ns;
+  cudaStream_t stream;
+};
+
+int launch_decode(const DecodeLaunch& a);
+
+}  // namespace bss

@@ -1,0 +1,144 @@
+/*
+ * Skip Softmax attention for NVIDIA B200 (sm_100a): C ABI of libattn.so.
+ *
+ * The operation is fused scaled-dot-product attention, softmax(Q K^T/sqrt(d)) V,
+ * evaluated block-wise (key tiles in ascending order, online softmax) with the
+ * Skip Softmax block-skip rule: a key tile is skipped -- its exponentials, its
+ * P*V product and its V load -- iff for EVERY query row of the row block the
+ * tile's local maximum score is strictly below that row's running maximum
+ * minus the threshold tau.  Source: "Accelerating Long-Context Inference with
+ * Skip Softmax in NVIDIA TensorRT-LLM", Key Points and Detailed Analysis (the
+ * page's comparison value is garbled in its transcript and is read as
+ * m_i - tau; tau is the user-set speed/accuracy knob of the same sections).
+ * Scores are S = Q K^T / sqrt(d) (natural-log units); tau is in those units.
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are bf16, contiguous, head dimension fastest:
+ *       Q, O  [B, Hq,  N, d]      K, V  [B, Hkv, N, d]     (prefill)
+ *       q, o  [B, Hq,  d]         K, V  [B, Hkv, L, d]     (decode)
+ *     Query head h reads KV head floor(h / (Hq/Hkv)) (grouped-query attention).
+ *   - Every tensor pointer is a DEVICE pointer on the current CUDA device,
+ *     16-byte aligned.  The caller owns all buffers; the library never frees
+ *     or keeps a caller pointer past the call's completion on the stream.
+ *   - tau >= 0; tau = +INFINITY gives exact attention (nothing is skipped).
+ *     NaN or negative tau is rejected.  Inputs must be finite.
+ *   - Calls are asynchronous on the stream they are given (the plain forms
+ *     use the stream set with attn_set_stream, default the legacy stream).
+ *     The returned status covers argument validation and launch errors only;
+ *     a kernel that gave up on a bounded internal wait is reported later by
+ *     attn_sync_status().
+ *   - There is no CPU fallback: without an sm_100 device every compute call
+ *     returns ATTN_ERR_UNSUPPORTED.
+ */
+#ifndef SKIP_SOFTMAX_ATTN_H
+#define SKIP_SOFTMAX_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_INVALID_ARG = 1, /* bad pointer, size, tau, tile or alignment   */
+  ATTN_ERR_UNSUPPORTED = 2, /* no sm_100 device, or a shape beyond limits  */
+  ATTN_ERR_CUDA = 3,        /* a CUDA runtime/driver call failed           */
+  ATTN_ERR_TIMEOUT = 4      /* a kernel gave up on a bounded wait          */
+} attn_status;
+
+/* Device status word values written by kernels that gave up (internal). */
+#define ATTN_DEVICE_TIMEOUT_BASE 0x100
+
+/*
+ * Prefill (self-attention over N tokens), Skip Softmax rule above.
+ *   causal   0: every query sees every key.  1: top-left aligned causal mask,
+ *            query i sees keys k <= i; key tiles wholly above the diagonal of
+ *            a row block are not visited.
+ *   Br, Bc   row-block and key-tile sizes of the skip rule:
+ *            (64,64), (128,64) or (128,128).  d in {64, 128}.
+ *   Errors: ATTN_ERR_INVALID_ARG for null/misaligned pointers, B/Hq/Hkv/N <= 0,
+ *   Hq % Hkv != 0, unsupported d/Br/Bc, NaN or negative tau.
+ */
+ATTN_API int attn_prefill(const void* Q, const void* K, const void* V, void* O, int B, int Hq, int Hkv,
+                 int N, int d, int causal, float tau, int Br, int Bc);
+
+/*
+ * As attn_prefill, on an explicit stream (a cudaStream_t passed as void*,
+ * NULL = legacy stream), optionally writing the skip decisions:
+ *   skip_mask  nullable device buffer uint8 [B, Hq, ceil(N/Br), ceil(N/Bc)]:
+ *              0 tile kept, 1 tile skipped, 2 tile not visited (causal).
+ */
+ATTN_API int attn_prefill_ex(const void* Q, const void* K, const void* V, void* O, int B, int Hq, int Hkv,
+                    int N, int d, int causal, float tau, int Br, int Bc, void* stream,
+                    uint8_t* skip_mask);
+
+/*
+ * Decode: one new query token per (batch, query head) against L cached keys,
+ * no mask.  The rows of the skip test are the g = Hq/Hkv query heads that
+ * share one KV head (they share the V tile that a skip avoids loading).  The
+ * key range of each (batch, KV head) is cut into splits of
+ * attn_decode_split_len(B, Hkv, L) keys; inside a split, tiles of 64 keys are
+ * visited in ascending order and the running maximum starts at -inf.  The
+ * split results are merged exactly (log-sum-exp).
+ * d in {64, 128}; g in {1, 2, 4, 8}.
+ * The plain form allocates (once, and grows when needed) a device workspace
+ * that attn_shutdown() frees.
+ */
+ATTN_API int attn_decode(const void* q, const void* K, const void* V, void* o, int B, int Hq, int Hkv,
+                int L, int d, float tau);
+
+/*
+ * As attn_decode on an explicit stream with a caller-provided workspace of at
+ * least attn_decode_workspace_bytes(B, Hq, Hkv, L, d) bytes (256-byte
+ * aligned device memory; ws may be NULL only if ws_bytes is 0, in which case
+ * the library's own workspace is used).  skip_mask: nullable device buffer
+ * uint8 [B, Hkv, ceil(L/64)] (0 kept, 1 skipped).
+ */
+ATTN_API int attn_decode_ex(const void* q, const void* K, const void* V, void* o, int B, int Hq, int Hkv,
+                   int L, int d, float tau, void* stream, uint8_t* skip_mask, void* ws,
+                   size_t ws_bytes);
+
+/* Split length in keys (a multiple of 64) used by decode: a deterministic
+ * function of (B, Hkv, L) only.  Returns -1 for non-positive arguments. */
+ATTN_API int attn_decode_split_len(int B, int Hkv, int L);
+
+/* Key-tile size of the decode skip test (64). */
+ATTN_API int attn_decode_tile(void);
+
+/* Workspace bytes attn_decode_ex needs; 0 for invalid arguments. */
+ATTN_API size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int L, int d);
+
+/* Stream used by the plain forms (cudaStream_t as void*; NULL = legacy). */
+ATTN_API int attn_set_stream(void* stream);
+
+/* Synchronise the current device, then report and clear the device status
+ * word: ATTN_OK, or ATTN_ERR_TIMEOUT if a kernel gave up on a bounded wait
+ * (attn_last_timeout_site() then names the wait), or ATTN_ERR_CUDA. */
+ATTN_API int attn_sync_status(void);
+
+/* Site code of the last wait that gave up (0 if none), for diagnostics. */
+ATTN_API int attn_last_timeout_site(void);
+
+/* Limit, in milliseconds, of every bounded wait inside the kernels
+ * (default 2000).  Values < 1 are rejected. */
+ATTN_API int attn_set_wait_limit_ms(int ms);
+
+/* Human-readable name of a status code (static string). */
+ATTN_API const char* attn_status_string(int status);
+
+/* Free the library-owned decode workspace on every device it was allocated. */
+ATTN_API void attn_shutdown(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SKIP_SOFTMAX_ATTN_H */
