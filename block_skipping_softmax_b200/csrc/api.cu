@@ -140,8 +140,12 @@ int attn_decode_split_len(int B, int Hkv, int L) {
   const long long slots = 296;
   const long long groups = static_cast<long long>(B) * Hkv;
   const long long n_tiles = (L + bss::kDecodeTile - 1) / bss::kDecodeTile;
+  // A split's running max starts at -inf, so its first tile is always kept:
+  // splits are at least 8 tiles (512 keys) long so that the skip test has a
+  // history to compare against.
+  const long long min_tps = n_tiles < 8 ? n_tiles : 8;
   long long best_tps = n_tiles, best_cost = -1;
-  for (long long tps = n_tiles; tps >= 1; --tps) {
+  for (long long tps = n_tiles; tps >= min_tps; --tps) {
     const long long ns = (n_tiles + tps - 1) / tps;
     if (ns > 4096) break;
     const long long waves = (groups * ns + slots - 1) / slots;

@@ -365,7 +365,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_ref = m_cand;
       }
       // P = 2^(x - m_ref) as bf16 pairs, written over this row's S columns
-      // (64 scores -> 32 packed columns per store)
+      // (64 scores -> 32 packed columns per store).  The row sum adds the
+      // bf16-rounded values that the P*V MMA multiplies, so numerator and
+      // denominator see the same weights and the rounding of a dominant
+      // weight cancels in O / l.
       float rs = 0.f;
 #pragma unroll
       for (int c0 = 0; c0 < BC; c0 += 64) {
@@ -375,8 +378,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           float p0 = ex2(x[c0 + 2 * c] - m_ref);
           float p1 = ex2(x[c0 + 2 * c + 1] - m_ref);
           if (!row_valid) p0 = p1 = 0.f;
-          rs += p0 + p1;
-          pk[c] = pack_bf16x2(p0, p1);
+          const uint32_t w = pack_bf16x2(p0, p1);
+          rs += __uint_as_float(w << 16) + __uint_as_float(w & 0xffff0000u);
+          pk[c] = w;
         }
         tmem_st32(tS(sb) + lane_off + c0 / 2, pk);
       }
