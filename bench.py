@@ -1,0 +1,415 @@
+"""Benchmark of Skip Softmax attention on B200 (prefill and decode).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl own|reference]
+
+One JSON line on stdout (rank 0).  Headline (``value``): prefill
+dense-equivalent TFLOP/s on the non-causal encoder workload
+(B=64, Hq=Hkv=32, N=512, d=128, Br=128, Bc=64, tau=inf) -- a step is one
+attn_prefill call over that batch, inputs resident in HBM.  The decode half
+of the metric (KV-read GB/s on B=16, Hq=32, Hkv=8, L=32768, d=128) is timed
+the same way and reported under ``decode``; the other workloads and
+thresholds are under ``workloads``.
+
+Timing: W untimed warm-up steps, then exactly K steps between two CUDA events
+on the launching stream, bracketed by a barrier and a device synchronise, max
+over ranks.  Every workload's inputs (>= 1.07 GB, or 168 MB for the 8B layer)
+are larger than the 126 MB L2, so consecutive steps do not hit in L2.
+Multi-GPU: every rank runs its own copy of the workload (independent
+sequences; no collective on the data path) -> weak scaling.
+
+``--impl reference`` times the fp64 CPU oracle (the deliberately slow
+reference program) on a bounded sample of the same workload, on this host's
+cores, in the same unit.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+MAIN = "encoder_64x32x512_d128"
+DECODE = "gqa_decode_16x32q8kv_L32768"
+METRIC = "prefill attn TFLOP/s (dense-equiv) & % tensor peak; decode KV-read GB/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def dense_flops(w):
+    f = 4.0 * w["B"] * w["Hq"] * w["N"] * w["N"] * w["d"]
+    return f / 2 if w["causal"] else f
+
+
+def compulsory_prefill_bytes(w):
+    return 2 * w["B"] * w["Hq"] * w["N"] * w["d"] * 2 + 2 * w["B"] * w["Hkv"] * w["N"] * w["d"] * 2
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 100 ms."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.rows = []
+        self.proc = None
+        self.gpu = gpu_index
+        self.t_start = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.rows.append((time.time(), [x.strip() for x in line.split(",")]))
+
+    def mark(self):
+        return time.time()
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self, t0=None, t1=None):
+        rows = [r for t, r in self.rows if (t0 is None or t >= t0) and (t1 is None or t <= t1)]
+        window = "timed region"
+        if len(rows) < 2:
+            rows = [r for _, r in self.rows]
+            window = "whole GPU phase"
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for name, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(rows), "window": window,
+                "power_w_max": max((float(r[3]) for r in rows if r[3].replace(".", "").isdigit()),
+                                   default=None)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def cpu_cores():
+    return len(os.sched_getaffinity(0))
+
+
+# --------------------------------------------------------------------------- CPU oracle
+def oracle_sample_rate(w, target_s, Q=None, K=None, V=None, seed=1):
+    """Time the fp64 oracle on a sample of row blocks of workload w (~target_s
+    of CPU work).  Returns (TFLOP/s, seconds, n_row_blocks, cores)."""
+    import numpy as np
+
+    import oracle
+    from block_skipping_softmax_b200 import inputs
+
+    if Q is None:
+        Q, K, V = inputs.prefill_inputs(w["B"], w["Hq"], w["Hkv"], w["N"], w["d"], seed=0, **w["gen"])
+    n_rb = -(-w["N"] // w["Br"])
+    rng = np.random.default_rng(seed)
+    all_units = [(b, h, rb) for b in range(w["B"]) for h in range(w["Hq"]) for rb in range(n_rb)]
+    cores = cpu_cores()
+
+    def flops_of(units):
+        f = 0.0
+        for _, _, rb in units:
+            rows = min(w["N"], (rb + 1) * w["Br"]) - rb * w["Br"]
+            keys = min(w["N"], (rb + 1) * w["Br"]) if w["causal"] else w["N"]
+            f += 4.0 * rows * keys * w["d"] * (0.5 if w["causal"] else 1.0)
+        return f
+
+    def run(units):
+        t = time.perf_counter()
+        oracle.prefill(Q, K, V, w["causal"], math.inf, w["Br"], w["Bc"], units=units,
+                       want_exact=False, nthreads=cores)
+        return time.perf_counter() - t
+
+    n = min(len(all_units), max(cores, 8))
+    pick = [all_units[i] for i in rng.choice(len(all_units), n, replace=False)]
+    t = run(pick)
+    n2 = int(min(len(all_units), max(n, n * target_s / max(t, 1e-3))))
+    pick = [all_units[i] for i in rng.choice(len(all_units), n2, replace=False)]
+    t = run(pick)
+    return flops_of(pick) / t / 1e12, t, n2, cores
+
+
+def reference_arm(args, world, rank):
+    if rank != 0:
+        return 0
+    from block_skipping_softmax_b200 import inputs
+
+    w = inputs.WORKLOADS[MAIN]
+    Q, K, V = inputs.prefill_inputs(w["B"], w["Hq"], w["Hkv"], w["N"], w["d"], seed=0, **w["gen"])
+    # each step: a fresh sample of row blocks sized to ~1.5 s of CPU time
+    rates, secs = [], []
+    for i in range(args.warmup + args.steps):
+        r, t, n, cores = oracle_sample_rate(w, 1.5, Q, K, V, seed=100 + i)
+        if i >= args.warmup:
+            rates.append(r)
+            secs.append(t)
+    value = statistics.mean(rates)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * statistics.mean(secs),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": MAIN, "B": w["B"], "Hq": w["Hq"], "Hkv": w["Hkv"], "N": w["N"],
+                   "d": w["d"], "causal": w["causal"], "Br": w["Br"], "Bc": w["Bc"], "tau": "inf"},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{n} random row blocks of {w['Br']} queries per step (of "
+                                   f"{w['B'] * w['Hq'] * (-(-w['N'] // w['Br']))})"},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------------- GPU arm
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="own", choices=["own", "reference"])
+    ap.add_argument("--quick", action="store_true", help="skip the extra workloads and the CPU baseline")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    world, rank, local = dist_setup()
+
+    if args.impl == "reference":
+        return reference_arm(args, world, rank)
+
+    import torch
+
+    import block_skipping_softmax_b200 as bss
+    from block_skipping_softmax_b200 import build as bss_build
+    from block_skipping_softmax_b200 import inputs
+
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    if rank == 0:
+        bss_build.build()
+    if dist:
+        dist.barrier()
+    bss.lib()
+    peaks, peak_src = load_peaks()
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if dist:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if not dist:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def timed(fn, steps, warmup):
+        for _ in range(warmup):
+            fn()
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0 = time.time()
+        e0.record(stream)
+        for _ in range(steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        t1 = time.time()
+        barrier()
+        st = bss.attn_sync_status()
+        if st != 0:
+            raise RuntimeError(f"kernel status {bss.attn_status_string(st)}")
+        return max_over_ranks(e0.elapsed_time(e1) / steps), t0, t1
+
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
+    clocks = ClockSampler(int(vis[local]) if local < len(vis) and vis[local].strip().isdigit() else local)
+    if rank == 0:
+        clocks.start()
+
+    # ---------------- headline: prefill, encoder workload, tau = inf
+    w = inputs.WORKLOADS[MAIN]
+    Qm, Km, Vm = inputs.prefill_inputs(w["B"], w["Hq"], w["Hkv"], w["N"], w["d"], seed=rank, **w["gen"])
+    Q, K, V = Qm.to(dev), Km.to(dev), Vm.to(dev)
+    O = torch.empty_like(Q)
+
+    def step():
+        bss.prefill(Q, K, V, w["causal"], math.inf, w["Br"], w["Bc"], out=O)
+
+    ms, t0, t1 = timed(step, args.steps, args.warmup)
+    flops = dense_flops(w)
+    value = world * flops / (ms * 1e-3) / 1e12
+    achieved = flops / (ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                "peak_source": f"{peak_src} bf16 burst (kernel timed alone)",
+                "kernel": "prefill_kernel<128,128,64,false>",
+                "algorithmic": "4*B*Hq*N^2*d dense-equivalent FLOPs per launch"}
+    clk = clocks.summary(t0, t1) if rank == 0 else None
+
+    # ---------------- end to end through the public API from pinned host memory
+    Qp, Kp, Vp = Qm.pin_memory(), Km.pin_memory(), Vm.pin_memory()
+    Op = torch.empty_like(Qm).pin_memory()
+
+    def e2e_step():
+        Q.copy_(Qp, non_blocking=True)
+        K.copy_(Kp, non_blocking=True)
+        V.copy_(Vp, non_blocking=True)
+        bss.prefill(Q, K, V, w["causal"], math.inf, w["Br"], w["Bc"], out=O)
+        Op.copy_(O, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 20))
+    ms_e2e, _, _ = timed(e2e_step, e2e_steps, 2)
+    e2e = {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+           "h2d_bytes_per_step": Qp.numel() * 2 + Kp.numel() * 2 + Vp.numel() * 2,
+           "d2h_bytes_per_step": Op.numel() * 2, "ms_per_step": ms_e2e,
+           "path": "pinned host -> cudaMemcpyAsync -> attn_prefill_ex -> pinned host"}
+    del Qp, Kp, Vp, Op
+
+    # tau = 4 on the same workload, plus its skipped fraction
+    extras = {}
+
+    def prefill_extra(name, wl, Qd, Kd, Vd, tau, steps, warmup):
+        Od = torch.empty_like(Qd)
+        ms_x, _, _ = timed(lambda: bss.prefill(Qd, Kd, Vd, wl["causal"], tau, wl["Br"], wl["Bc"], out=Od),
+                           steps, warmup)
+        _, mask = bss.prefill(Qd, Kd, Vd, wl["causal"], tau, wl["Br"], wl["Bc"], out=Od, skip_mask=True)
+        mk = mask[mask != 2]
+        f = dense_flops(wl)
+        skipped = float((mk == 1).float().mean().item())
+        visited = mk.numel()
+        # executed MMA FLOPs: every visited tile's QK^T, every kept tile's PV
+        executed = visited * 2.0 * wl["Br"] * wl["Bc"] * wl["d"] * (2.0 - skipped)
+        extras[f"{name}@tau={tau}"] = {
+            "ms": ms_x, "dense_tflops": f / (ms_x * 1e-3) / 1e12,
+            "executed_tflops": executed / (ms_x * 1e-3) / 1e12,
+            "frac_of_peak": f / (ms_x * 1e-3) / 1e12 / peaks["bf16_tflops"],
+            "skipped_fraction": skipped, "tiles_visited": visited}
+
+    prefill_extra(MAIN, w, Q, K, V, math.inf, 3, 1)
+    prefill_extra(MAIN, w, Q, K, V, 4.0, max(3, args.steps // 4), 2)
+    del Q, K, V, O
+    torch.cuda.empty_cache()
+
+    # ---------------- decode: KV-read GB/s
+    wd = inputs.WORKLOADS[DECODE]
+    qh, Kh, Vh = inputs.decode_inputs(wd["B"], wd["Hq"], wd["Hkv"], wd["L"], wd["d"], seed=rank, **wd["gen"])
+    q, Kd, Vd = qh.to(dev), Kh.to(dev), Vh.to(dev)
+    del Kh, Vh
+    o = torch.empty_like(q)
+    decode = {}
+    kv_bytes = wd["B"] * wd["Hkv"] * wd["L"] * wd["d"] * 2
+    for tau in wd["taus"]:
+        ms_d, d0, d1 = timed(lambda: bss.decode(q, Kd, Vd, tau, out=o), args.steps, args.warmup)
+        _, mask = bss.decode(q, Kd, Vd, tau, out=o, skip_mask=True)
+        kept = 1.0 - float((mask == 1).float().mean().item())
+        read = kv_bytes * (1.0 + kept)
+        gbs = read / (ms_d * 1e-3) / 1e9
+        decode[f"tau={tau}"] = {
+            "value": world * gbs, "unit": "GB/s", "ms_per_step": ms_d, "latency_us": ms_d * 1000,
+            "dense_equiv_gbs": world * 2 * kv_bytes / (ms_d * 1e-3) / 1e9,
+            "skipped_fraction": 1.0 - kept, "gpu_launches": 2 * args.steps,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                         "peak_source": f"{peak_src} HBM copy bandwidth",
+                         "kernel": "decode_partial_kernel<128,4> + decode_combine_kernel<128>",
+                         "algorithmic": "K bytes + kept fraction x V bytes per launch"},
+            "split_len": bss.attn_decode_split_len(wd["B"], wd["Hkv"], wd["L"])}
+    del q, Kd, Vd, o
+    torch.cuda.empty_cache()
+
+    # ---------------- the causal LLM-layer workloads (timing inputs drawn on the GPU)
+    if not args.quick:
+        for name, steps in (("llama3_8b_causal_N8192", max(3, args.steps // 4)),
+                            ("llama33_70b_causal_N131072", 3)):
+            wl = inputs.WORKLOADS[name]
+            Qd, Kd2, Vd2 = inputs.prefill_inputs(wl["B"], wl["Hq"], wl["Hkv"], wl["N"], wl["d"], seed=rank,
+                                                 device=str(dev), **wl["gen"])
+            for tau in wl["taus"]:
+                prefill_extra(name, wl, Qd, Kd2, Vd2, tau, steps, 1)
+            del Qd, Kd2, Vd2
+            torch.cuda.empty_cache()
+    if rank == 0:
+        clocks.stop()
+
+    cpu_base = None
+    if rank == 0 and world == 1 and not args.quick:
+        r, t, n, cores = oracle_sample_rate(w, 10.0, Qm, Km, Vm)
+        cpu_base = {"value": r, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                    "sample": f"{n} random row blocks ({w['Br']} queries x {w['N']} keys each) of "
+                              f"{MAIN}, {t:.1f} s of fp64 CPU work"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": MAIN, "B": w["B"], "Hq": w["Hq"], "Hkv": w["Hkv"], "N": w["N"],
+                       "d": w["d"], "causal": w["causal"], "Br": w["Br"], "Bc": w["Bc"], "tau": "inf",
+                       "parallelism": f"replicas x{world} (independent sequences)",
+                       "l2": "inputs 1.07 GB per step > 126 MB L2 (no flush needed)"},
+            "roofline": roofline, "frac_of_tensor_peak": achieved / peaks["bf16_tflops"],
+            "e2e": e2e, "gpu_launches": args.steps, "clocks": clk, "cpu_baseline": cpu_base,
+            "decode": {"metric": "decode KV-read GB/s", "workload": DECODE, **decode},
+            "workloads": extras,
+        }
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

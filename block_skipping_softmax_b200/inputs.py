@@ -2,8 +2,11 @@
 
 This module holds no attention arithmetic: it only draws Gaussian tensors and
 places the "attention sink" rows, so that the CUDA path, the tests and the
-bench all see bit-identical bf16 inputs.  All draws happen on the CPU with
-``torch.Generator`` (deterministic for a given torch build).
+bench all see bit-identical bf16 inputs.  Draws happen on the CPU with
+``torch.Generator`` (deterministic for a given torch build).  With
+``device="cuda"`` the same recipe is drawn by the GPU's generator instead
+(same distribution, different bits): the bench uses that only to time very
+large workloads whose CPU draw would take minutes.
 
 Recipe (one line per knob):
   * every (tensor, batch, head) gets its own seed ``derive(seed, tag, b, h)``;
@@ -38,10 +41,10 @@ def derive(seed: int, tag: str, b: int = 0, h: int = 0) -> int:
     return x & ((1 << 63) - 1)
 
 
-def _randn(rows: int, d: int, seed: int) -> torch.Tensor:
-    g = torch.Generator(device="cpu")
+def _randn(rows: int, d: int, seed: int, device: str = "cpu") -> torch.Tensor:
+    g = torch.Generator(device=device)
     g.manual_seed(seed)
-    return torch.randn(rows, d, generator=g, dtype=torch.float32)
+    return torch.randn(rows, d, generator=g, dtype=torch.float32, device=device)
 
 
 def unit_vector(d: int, seed: int) -> torch.Tensor:
@@ -51,7 +54,7 @@ def unit_vector(d: int, seed: int) -> torch.Tensor:
 
 def _par_map(fn, items, workers: int = 0):
     items = list(items)
-    if len(items) <= 1:
+    if len(items) <= 1 or workers == 1:
         return [fn(i) for i in items]
     import os
 
@@ -62,22 +65,22 @@ def _par_map(fn, items, workers: int = 0):
 
 def prefill_inputs(B: int, Hq: int, Hkv: int, N: int, d: int, *, seed: int = 0,
                    q_sigma: float = 1.0, q_u: float = 0.0, sink_scale: float | None = None,
-                   n_sinks: int = 4, q_heads=None):
+                   n_sinks: int = 4, q_heads=None, device: str = "cpu"):
     """Q [B,Hq,N,d], K, V [B,Hkv,N,d] bf16 on the CPU.
 
     ``q_heads``: optional iterable of (b, h) pairs; only those query heads are
     drawn (the others stay zero), which lets very long workloads be checked on
     a sample of heads without drawing all of Q.
     """
-    u = unit_vector(d, seed)
-    Q = torch.zeros(B, Hq, N, d, dtype=torch.bfloat16)
-    K = torch.empty(B, Hkv, N, d, dtype=torch.bfloat16)
-    V = torch.empty(B, Hkv, N, d, dtype=torch.bfloat16)
+    u = unit_vector(d, seed).to(device)
+    Q = torch.zeros(B, Hq, N, d, dtype=torch.bfloat16, device=device)
+    K = torch.empty(B, Hkv, N, d, dtype=torch.bfloat16, device=device)
+    V = torch.empty(B, Hkv, N, d, dtype=torch.bfloat16, device=device)
     qh = [(b, h) for b in range(B) for h in range(Hq)] if q_heads is None else list(q_heads)
 
     def make_q(bh):
         b, h = bh
-        z = _randn(N, d, derive(seed, "q", b, h))
+        z = _randn(N, d, derive(seed, "q", b, h), device)
         x = z * q_sigma
         if q_u:
             x = x + q_u * u
@@ -85,14 +88,15 @@ def prefill_inputs(B: int, Hq: int, Hkv: int, N: int, d: int, *, seed: int = 0,
 
     def make_kv(bh):
         b, h = bh
-        k = _randn(N, d, derive(seed, "k", b, h))
+        k = _randn(N, d, derive(seed, "k", b, h), device)
         if sink_scale is not None and n_sinks > 0:
             k[: min(n_sinks, N)] = sink_scale * math.sqrt(d) * u
         K[b, h] = k.to(torch.bfloat16)
-        V[b, h] = _randn(N, d, derive(seed, "v", b, h)).to(torch.bfloat16)
+        V[b, h] = _randn(N, d, derive(seed, "v", b, h), device).to(torch.bfloat16)
 
-    _par_map(make_q, qh)
-    _par_map(make_kv, [(b, h) for b in range(B) for h in range(Hkv)])
+    workers = 1 if device != "cpu" else 0
+    _par_map(make_q, qh, workers)
+    _par_map(make_kv, [(b, h) for b in range(B) for h in range(Hkv)], workers)
     return Q, K, V
 
 
