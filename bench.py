@@ -24,6 +24,7 @@ cores, in the same unit.
 from __future__ import annotations
 
 import argparse
+import gc
 import json
 import math
 import os
@@ -50,6 +51,28 @@ def load_peaks():
         return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
     except Exception:
         return dict(FALLBACK_PEAKS), "fallback"
+
+
+def measured_traffic(kernel: str, cu_file: str):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel's source changed since the counters were taken."""
+    import hashlib
+
+    csrc = os.path.join(ROOT, "block_skipping_softmax_b200", "csrc")
+    h = hashlib.sha256()
+    for f in (cu_file, "ptx.cuh", "kernels.cuh"):
+        with open(os.path.join(csrc, f), "rb") as fh:
+            h.update(fh.read())
+    digest = h.hexdigest()[:16]
+    try:
+        with open(os.path.join(ROOT, "profiles", "ncu_traffic.txt")) as fh:
+            for line in fh:
+                parts = line.split()
+                if len(parts) >= 3 and not line.startswith("#") and parts[0] == kernel and parts[1] == digest:
+                    return int(parts[2])
+    except OSError:
+        pass
+    return None
 
 
 def dense_flops(w):
@@ -124,10 +147,9 @@ class ClockSampler:
 
 
 def dist_setup():
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    return world, rank, local
+    from block_skipping_softmax_b200.replicas import rank_info
+
+    return rank_info()
 
 
 def cpu_cores():
@@ -164,13 +186,20 @@ def oracle_sample_rate(w, target_s, Q=None, K=None, V=None, seed=1):
                        want_exact=False, nthreads=cores)
         return time.perf_counter() - t
 
+    # calibrate: grow the sample until it takes a quarter of the target time
     n = min(len(all_units), max(cores, 8))
-    pick = [all_units[i] for i in rng.choice(len(all_units), n, replace=False)]
-    t = run(pick)
+    run(all_units[:n])  # first call pays for thread start-up
+    while True:
+        pick = [all_units[i] for i in rng.choice(len(all_units), n, replace=False)]
+        t = run(pick)
+        if t >= target_s / 4 or n >= len(all_units):
+            break
+        n = min(len(all_units), n * 4)
     n2 = int(min(len(all_units), max(n, n * target_s / max(t, 1e-3))))
-    pick = [all_units[i] for i in rng.choice(len(all_units), n2, replace=False)]
-    t = run(pick)
-    return flops_of(pick) / t / 1e12, t, n2, cores
+    if n2 > n:
+        pick = [all_units[i] for i in rng.choice(len(all_units), n2, replace=False)]
+        t = run(pick)
+    return flops_of(pick) / t / 1e12, t, len(pick), cores
 
 
 def reference_arm(args, world, rank):
@@ -248,15 +277,15 @@ def main():
             dist.barrier()
 
     def max_over_ranks(x):
-        if not dist:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        from block_skipping_softmax_b200.replicas import max_over_ranks as mor
+
+        return mor(x, dev)
 
     def timed(fn, steps, warmup):
         for _ in range(warmup):
             fn()
+        gc.collect()
+        gc.disable()  # no collector pauses between the two events
         barrier()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -267,6 +296,7 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         t1 = time.time()
+        gc.enable()
         barrier()
         st = bss.attn_sync_status()
         if st != 0:
@@ -292,7 +322,9 @@ def main():
     value = world * flops / (ms * 1e-3) / 1e12
     achieved = flops / (ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops"], "traffic": None,
+                "frac": achieved / peaks["bf16_tflops"],
+                "traffic": measured_traffic("prefill_kernel", "prefill_sm100.cu"),
+                "algorithmic_bytes": compulsory_prefill_bytes(w),
                 "peak_source": f"{peak_src} bf16 burst (kernel timed alone)",
                 "kernel": "prefill_kernel<128,128,64,false>",
                 "algorithmic": "4*B*Hq*N^2*d dense-equivalent FLOPs per launch"}
@@ -361,7 +393,8 @@ def main():
             "dense_equiv_gbs": world * 2 * kv_bytes / (ms_d * 1e-3) / 1e9,
             "skipped_fraction": 1.0 - kept, "gpu_launches": 2 * args.steps,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                         "frac": gbs / peaks["hbm_gbs"],
+                         "traffic": measured_traffic("decode_partial_kernel", "decode_sm100.cu"),
                          "peak_source": f"{peak_src} HBM copy bandwidth",
                          "kernel": "decode_partial_kernel<128,4> + decode_combine_kernel<128>",
                          "algorithmic": "K bytes + kept fraction x V bytes per launch"},

@@ -114,12 +114,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work item: (row block, batch*head); causal row blocks run longest first
+  // ---- work item: (row block, batch*head).  Causal: the longest row blocks
+  // run first, heads fastest (the g heads of a KV group share K/V in L2).
+  // Non-causal: row blocks fastest, so the CTAs that read one head's K/V run
+  // together and the re-reads hit L2.
   const int n_rb = (N + BR - 1) / BR;
   const int BH = B * Hq;
-  const int bh = blockIdx.x % BH;
-  const int rb_lin = blockIdx.x / BH;
-  const int rb = CAUSAL ? (n_rb - 1 - rb_lin) : rb_lin;
+  const int bh = CAUSAL ? static_cast<int>(blockIdx.x % BH) : static_cast<int>(blockIdx.x / n_rb);
+  const int rb = CAUSAL ? (n_rb - 1 - static_cast<int>(blockIdx.x / BH))
+                        : static_cast<int>(blockIdx.x % n_rb);
   const int b = bh / Hq;
   const int h = bh % Hq;
   const int g = Hq / Hkv;
