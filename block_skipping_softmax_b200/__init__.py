@@ -19,6 +19,7 @@ import os
 
 __all__ = [
     "AttnError", "lib", "attn_prefill", "attn_prefill_ex", "attn_decode", "attn_decode_ex",
+    "attn_decode_noalloc",
     "attn_decode_split_len", "attn_decode_tile", "attn_decode_workspace_bytes",
     "attn_set_stream", "attn_sync_status", "attn_last_timeout_site", "attn_set_wait_limit_ms",
     "attn_status_string", "attn_shutdown", "prefill", "decode", "STATUS",
@@ -53,6 +54,7 @@ def lib() -> ctypes.CDLL:
         "attn_prefill_ex": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, ci, vp, vp]),
         "attn_decode": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf]),
         "attn_decode_ex": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, vp, vp, vp, sz]),
+        "attn_decode_noalloc": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, vp, vp]),
         "attn_decode_split_len": (ci, [ci, ci, ci]),
         "attn_decode_tile": (ci, []),
         "attn_decode_workspace_bytes": (sz, [ci, ci, ci, ci, ci]),
@@ -87,6 +89,11 @@ def attn_decode(q, K, V, o, B, Hq, Hkv, L, d, tau) -> int:
 
 def attn_decode_ex(q, K, V, o, B, Hq, Hkv, L, d, tau, stream=None, skip_mask=None, ws=None, ws_bytes=0) -> int:
     return lib().attn_decode_ex(q, K, V, o, B, Hq, Hkv, L, d, float(tau), stream, skip_mask, ws, ws_bytes)
+
+
+def attn_decode_noalloc(q, K, V, o, B, Hq, Hkv, L, d, tau, stream=None, skip_mask=None) -> int:
+    """Decode with the library's fixed scratch array: no device allocation."""
+    return lib().attn_decode_noalloc(q, K, V, o, B, Hq, Hkv, L, d, float(tau), stream, skip_mask)
 
 
 def attn_decode_split_len(B, Hkv, L) -> int:

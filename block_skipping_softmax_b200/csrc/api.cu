@@ -93,6 +93,13 @@ void decode_ws_layout(int B, int Hq, int n_splits, int d, size_t* o_bytes, size_
 
 }  // namespace
 
+namespace bss {
+// Current device (sm_100 checked) and its device status word, for entry
+// points defined in other files.
+int device_context(int* dev, int** status) { return device_ready(dev, status); }
+unsigned long long wait_limit_ns() { return g_wait_limit_ns; }
+}  // namespace bss
+
 extern "C" {
 
 int attn_prefill_ex(const void* Q, const void* K, const void* V, void* O, int B, int Hq, int Hkv,

@@ -106,6 +106,28 @@ ATTN_API int attn_decode_ex(const void* q, const void* K, const void* V, void* o
                    int L, int d, float tau, void* stream, uint8_t* skip_mask, void* ws,
                    size_t ws_bytes);
 
+/*
+ * Decode that allocates nothing, for callers that cannot allocate device
+ * memory (a serving engine that has reserved all of HBM for its own pools, a
+ * latency-critical loop that must not meet the implicit synchronisation of
+ * cudaMalloc/cudaFree, a minimal binding that can only pass q, K, V and o).
+ * The pages have no counterpart: this is a deployment variant of attn_decode.
+ *   Same arguments, layouts and results as attn_decode_ex; the per-split
+ *   scratch lives in a fixed 16 MiB array in device global memory, reserved
+ *   on every GPU that loads the library and kept until the process exits.
+ *   The first call on a device looks up that array's device address; make
+ *   that first call before any stream capture.  Every call shares the array
+ *   and leaves its contents behind (nothing in it needs clearing: each entry
+ *   read is written earlier in the same call), so calls that overlap on the
+ *   GPU -- on different streams, or from different threads -- race.
+ *   Errors: as attn_decode_ex, plus ATTN_ERR_UNSUPPORTED when the problem
+ *   needs more than 16 MiB of scratch (about B*Hq*splits*(d+1)*4 bytes).
+ *   Calls no cudaMalloc, cudaFree or allocating library routine.
+ */
+ATTN_API int attn_decode_noalloc(const void* q, const void* K, const void* V, void* o, int B,
+                                 int Hq, int Hkv, int L, int d, float tau, void* stream,
+                                 uint8_t* skip_mask);
+
 /* Split length in keys (a multiple of 64) used by decode: a deterministic
  * function of (B, Hkv, L) only.  Returns -1 for non-positive arguments. */
 ATTN_API int attn_decode_split_len(int B, int Hkv, int L);
