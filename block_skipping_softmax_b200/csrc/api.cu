@@ -130,7 +130,7 @@ int attn_prefill_ex(const void* Q, const void* K, const void* V, void* O, int B,
   a.status = status;
   a.wait_limit_ns = g_wait_limit_ns;
   a.stream = static_cast<cudaStream_t>(stream);
-  return bss::launch_prefill(a);
+  return Br == 128 ? bss::launch_prefill_pp(a) : bss::launch_prefill(a);
 }
 
 int attn_prefill(const void* Q, const void* K, const void* V, void* O, int B, int Hq, int Hkv,

@@ -25,7 +25,8 @@ struct PrefillLaunch {
   cudaStream_t stream;
 };
 
-int launch_prefill(const PrefillLaunch& a);
+int launch_prefill(const PrefillLaunch& a);     // one row block per CTA (any Br)
+int launch_prefill_pp(const PrefillLaunch& a);  // two row blocks per CTA, Br = 128
 
 constexpr int kDecodeTile = 64;  // keys per decode tile
 

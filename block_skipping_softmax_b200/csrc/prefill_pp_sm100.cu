@@ -1,0 +1,637 @@
+// Skip Softmax prefill for sm_100a, two row blocks per CTA ("ping-pong"),
+// persistent over work items.  Used for Br = 128.
+//
+// Method: "Accelerating Long-Context Inference with Skip Softmax in NVIDIA
+// TensorRT-LLM" (Key Points; Detailed Analysis): key tiles in ascending
+// order; tile j of a row block is skipped -- no exponentials, no P*V MMA --
+// iff every row of that row block has tile max < running max - tau.  The V
+// tile is loaded iff at least one of the CTA's two row blocks keeps it.
+//
+// Layout of one CTA (384 threads, one per SM, persistent):
+//   warpgroup 0: warp 0 TMA Q (both tiles) + K ring; warp 1 TMEM allocator
+//                and the single MMA-issuing thread; warp 2 TMA V ring
+//                (gated by the skip decisions); warp 3 idle.  56 registers.
+//   warpgroup 1: softmax of row block 0 (thread r owns row r).  224 registers.
+//   warpgroup 2: softmax of row block 1.                        224 registers.
+// TMEM (512 columns): O0 | O1 | S0 | S1, with P_t (bf16) written over S_t.
+// MMA issue order per key tile j:   PV0_j, S0_{j+1}, PV1_j, S1_{j+1}
+// so the exponentials of one row block overlap the other block's MMAs.  A
+// completed S_t_{j+1} implies PV_t_j completed (one thread issues them in
+// order), so softmax t may rescale O_t in TMEM without any further wait.
+// Every wait is bounded; a wait that gives up records a status code and the
+// CTA unwinds (leaving no copy or MMA in flight and freeing TMEM).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "kernels.cuh"
+#include "ptx.cuh"
+
+namespace bss {
+
+namespace {
+
+constexpr int kPPThreads = 384;
+constexpr int kPPRegs = 168;       // registers per thread at launch (checked on the host)
+constexpr int kProducerRegs = 56;  // 128 x 56 + 256 x 224 = 384 x 168
+constexpr int kSoftmaxRegs = 224;
+constexpr int kRows = 128;         // rows per tile (row block)
+constexpr int kDR = 4;             // decision ring
+constexpr float kRescale = 8.0f;   // lazy rescale threshold (log2 units)
+
+template <int D, int BC>
+struct PPCfg {
+  static constexpr int kPanels = D / 64;
+  static constexpr int kQTile = kRows * D * 2;
+  static constexpr int kQPanel = kRows * 128;
+  static constexpr int kKVBytes = BC * D * 2;
+  static constexpr int kKVPanel = BC * 128;
+  static constexpr int kKS = (BC == 128 && D == 128) ? 2 : 3;
+  static constexpr int kVS = (BC == 128 && D == 128) ? 2 : 3;
+  static constexpr int kOffQ = 0;                                 // two Q tiles
+  static constexpr int kOffK = kOffQ + 2 * kQTile;
+  static constexpr int kOffV = kOffK + kKS * kKVBytes;
+  static constexpr int kOffBar = kOffV + kVS * kKVBytes;
+  // q_full, q_empty, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS],
+  // s_full[2], p_full[2], o_full[2], dec_full[2][DR]
+  static constexpr int kNumBars = 2 + 2 * kKS + 2 * kVS + 6 + 2 * kDR;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffMisc + 256 + 1024;
+  static constexpr int kTmemCols = 512;
+  static_assert(2 * D + 2 * BC <= 512, "TMEM budget");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+};
+
+struct PPMisc {
+  uint32_t tmem_base;
+  int abort;
+  int dec[2][kDR];
+  int vote[2][2][4];
+};
+
+__device__ __forceinline__ void named_bar(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+template <int N>
+__device__ __forceinline__ void reg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void reg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
+__device__ __forceinline__ void pp_give_up(PPMisc* m, int* status, int where) {
+  reinterpret_cast<volatile int*>(&m->abort)[0] = 1;
+  atomicCAS(status, 0, ATTN_DEVICE_TIMEOUT_BASE + 32 + where);
+}
+
+// Work item -> (bh, pair).  Causal: longest pairs first, heads fastest.
+// Non-causal: pairs fastest, so CTAs reading one head's K/V run together.
+struct Item {
+  int bh, rb0, T0, T1, Tmax;  // T1 = 0 when the second row block does not exist
+};
+
+template <int BC, bool CAUSAL>
+__device__ __forceinline__ Item make_item(long long idx, int BH, int n_pairs, int n_rb, int N) {
+  Item it;
+  int pair;
+  if (CAUSAL) {
+    pair = n_pairs - 1 - static_cast<int>(idx / BH);
+    it.bh = static_cast<int>(idx % BH);
+  } else {
+    pair = static_cast<int>(idx % n_pairs);
+    it.bh = static_cast<int>(idx / n_pairs);
+  }
+  it.rb0 = 2 * pair;
+  const int n_tiles = (N + BC - 1) / BC;
+  auto visited = [&](int rb) {
+    const int last = min(N, (rb + 1) * kRows) - 1;
+    return CAUSAL ? (last / BC + 1) : n_tiles;
+  };
+  it.T0 = visited(it.rb0);
+  it.T1 = (it.rb0 + 1 < n_rb) ? visited(it.rb0 + 1) : 0;
+  it.Tmax = max(it.T0, it.T1);
+  return it;
+}
+
+}  // namespace
+
+template <int D, int BC, bool CAUSAL>
+__global__ void __launch_bounds__(kPPThreads, 1)
+    prefill_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                      const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ O,
+                      uint8_t* __restrict__ skip_mask, int* __restrict__ status, int B, int Hq,
+                      int Hkv, int N, float scale_log2, float tau_log2, int tau_is_inf,
+                      unsigned long long wait_limit_ns) {
+  using C = PPCfg<D, BC>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const uint32_t sQ = sbase + C::kOffQ;
+  const uint32_t sK = sbase + C::kOffK;
+  const uint32_t sV = sbase + C::kOffV;
+  const uint32_t bar0 = sbase + C::kOffBar;
+  const uint32_t b_q_full = bar0, b_q_empty = bar0 + 8;
+  auto b_k_full = [&](int s) { return bar0 + 8u * (2 + s); };
+  auto b_k_empty = [&](int s) { return bar0 + 8u * (2 + C::kKS + s); };
+  auto b_v_full = [&](int s) { return bar0 + 8u * (2 + 2 * C::kKS + s); };
+  auto b_v_empty = [&](int s) { return bar0 + 8u * (2 + 2 * C::kKS + C::kVS + s); };
+  constexpr int kB = 2 + 2 * C::kKS + 2 * C::kVS;
+  auto b_s_full = [&](int t) { return bar0 + 8u * (kB + t); };
+  auto b_p_full = [&](int t) { return bar0 + 8u * (kB + 2 + t); };
+  auto b_o_full = [&](int t) { return bar0 + 8u * (kB + 4 + t); };
+  auto b_dec = [&](int t, int i) { return bar0 + 8u * (kB + 6 + t * kDR + i); };
+  PPMisc* misc = reinterpret_cast<PPMisc*>(smem + C::kOffMisc);
+  volatile int* abort_flag = &misc->abort;
+  volatile int* vdec = &misc->dec[0][0];
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n_rb = (N + kRows - 1) / kRows;
+  const int n_pairs = (n_rb + 1) / 2;
+  const int BH = B * Hq;
+  const int g = Hq / Hkv;
+  const int n_tiles = (N + BC - 1) / BC;
+  const long long n_items = static_cast<long long>(BH) * n_pairs;
+
+  if (threadIdx.x == 0) {
+    mbar_init(b_q_full, 1);
+    mbar_init(b_q_empty, 1);
+    for (int s = 0; s < C::kKS; ++s) {
+      mbar_init(b_k_full(s), 1);
+      mbar_init(b_k_empty(s), 1);
+    }
+    for (int s = 0; s < C::kVS; ++s) {
+      mbar_init(b_v_full(s), 1);
+      mbar_init(b_v_empty(s), 1);
+    }
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(b_s_full(t), 1);
+      mbar_init(b_p_full(t), 4);
+      mbar_init(b_o_full(t), 1);
+      for (int i = 0; i < kDR; ++i) mbar_init(b_dec(t, i), 1);
+    }
+    misc->abort = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&misc->tmem_base), C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc->tmem_base;
+  auto tO = [&](int t) { return tmem + t * D; };
+  auto tS = [&](int t) { return tmem + 2 * D + t * BC; };
+
+  if (warp < 4) {
+    reg_dec<kProducerRegs>();
+    if (warp == 0 && lane == 0) {
+      // ---------------------------------------------------- Q and K producer
+      int kload = 0, items = 0, kdone = 0;
+      bool alive = true;
+      for (long long idx = blockIdx.x; alive && idx < n_items; idx += gridDim.x, ++items) {
+        const Item it = make_item<BC, CAUSAL>(idx, BH, n_pairs, n_rb, N);
+        const int bkv = (it.bh / Hq) * Hkv + (it.bh % Hq) / g;
+        if (items > 0 &&
+            !mbar_wait(b_q_empty, (items - 1) & 1, abort_flag, wait_limit_ns)) {
+          pp_give_up(misc, status, 1);
+          break;
+        }
+        const int nq = it.T1 > 0 ? 2 : 1;
+        mbar_arrive_expect_tx(b_q_full, nq * C::kQTile);
+        for (int t = 0; t < nq; ++t)
+          for (int p = 0; p < C::kPanels; ++p)
+            tma_load_3d(sQ + t * C::kQTile + p * C::kQPanel, &tmQ, b_q_full, p * 64,
+                        (it.rb0 + t) * kRows, it.bh);
+        for (int j = 0; j < it.Tmax; ++j) {
+          const int s = kload % C::kKS;
+          if (kload >= C::kKS &&
+              !mbar_wait(b_k_empty(s), ((kload / C::kKS) - 1) & 1, abort_flag, wait_limit_ns)) {
+            pp_give_up(misc, status, 2);
+            alive = false;
+            break;
+          }
+          mbar_arrive_expect_tx(b_k_full(s), C::kKVBytes);
+          for (int p = 0; p < C::kPanels; ++p)
+            tma_load_3d(sK + s * C::kKVBytes + p * C::kKVPanel, &tmK, b_k_full(s), p * 64, j * BC,
+                        bkv);
+          ++kload;
+        }
+        kdone = items + 1;
+      }
+      // never leave with a copy in flight
+      if (kdone > 0) mbar_drain(b_q_full, (kdone - 1) & 1, wait_limit_ns);
+      for (int t = max(0, kload - C::kKS); t < kload; ++t)
+        mbar_drain(b_k_full(t % C::kKS), (t / C::kKS) & 1, wait_limit_ns);
+    } else if (warp == 2 && lane == 0) {
+      // ---------------------------------------------------- V producer
+      int vload = 0;
+      int dl[2] = {0, 0};
+      bool alive = true;
+      auto issue_v = [&](int j, int bkv) -> bool {
+        const int s = vload % C::kVS;
+        if (vload >= C::kVS &&
+            !mbar_wait(b_v_empty(s), ((vload / C::kVS) - 1) & 1, abort_flag, wait_limit_ns))
+          return false;
+        mbar_arrive_expect_tx(b_v_full(s), C::kKVBytes);
+        for (int p = 0; p < C::kPanels; ++p)
+          tma_load_3d(sV + s * C::kKVBytes + p * C::kKVPanel, &tmV, b_v_full(s), p * 64, j * BC, bkv);
+        ++vload;
+        return true;
+      };
+      for (long long idx = blockIdx.x; alive && idx < n_items; idx += gridDim.x) {
+        const Item it = make_item<BC, CAUSAL>(idx, BH, n_pairs, n_rb, N);
+        const int bkv = (it.bh / Hq) * Hkv + (it.bh % Hq) / g;
+        const int T[2] = {it.T0, it.T1};
+        for (int j = 0; alive && j < it.Tmax; ++j) {
+          if (tau_is_inf) {
+            if (!issue_v(j, bkv)) {
+              pp_give_up(misc, status, 4);
+              alive = false;
+            }
+            continue;
+          }
+          // V_j is loaded as soon as either row block keeps tile j; every
+          // decision is still consumed, in order
+          bool issued = false;
+          for (int t = 0; alive && t < 2; ++t) {
+            if (j >= T[t]) continue;
+            const int di = dl[t] % kDR;
+            if (!mbar_wait(b_dec(t, di), (dl[t] / kDR) & 1, abort_flag, wait_limit_ns)) {
+              pp_give_up(misc, status, 3);
+              alive = false;
+              break;
+            }
+            ++dl[t];
+            if (vdec[t * kDR + di] && !issued) {
+              if (!issue_v(j, bkv)) {
+                pp_give_up(misc, status, 4);
+                alive = false;
+                break;
+              }
+              issued = true;
+            }
+          }
+        }
+      }
+      for (int t = max(0, vload - C::kVS); t < vload; ++t)
+        mbar_drain(b_v_full(t % C::kVS), (t / C::kVS) & 1, wait_limit_ns);
+    } else if (warp == 1 && lane == 0) {
+      // ---------------------------------------------------- MMA issuer
+      constexpr uint32_t idS = idesc_bf16_f32(kRows, BC, false, false);
+      constexpr uint32_t idPV = idesc_bf16_f32(kRows, D, false, true);
+      int kuse = 0, vuse = 0, items = 0;
+      int pc[2] = {0, 0}, dc[2] = {0, 0};
+      bool alive = true;
+      auto issue_S = [&](int t, int kslot) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk & 3) * 32;
+          const uint64_t da = sw128_desc(sQ + t * C::kQTile + (kk >> 2) * C::kQPanel + off, 16, 1024);
+          const uint64_t db =
+              sw128_desc(sK + kslot * C::kKVBytes + (kk >> 2) * C::kKVPanel + off, 16, 1024);
+          mma_ss(tS(t), da, db, idS, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(b_s_full(t));
+      };
+      for (long long idx = blockIdx.x; alive && idx < n_items; idx += gridDim.x, ++items) {
+        const Item it = make_item<BC, CAUSAL>(idx, BH, n_pairs, n_rb, N);
+        const int T[2] = {it.T0, it.T1};
+        if (!mbar_wait(b_q_full, items & 1, abort_flag, wait_limit_ns)) {
+          pp_give_up(misc, status, 5);
+          break;
+        }
+        // prologue: S_t_0
+        if (!mbar_wait(b_k_full(kuse % C::kKS), (kuse / C::kKS) & 1, abort_flag, wait_limit_ns)) {
+          pp_give_up(misc, status, 6);
+          break;
+        }
+        tc_fence_after();
+        for (int t = 0; t < 2; ++t)
+          if (T[t] > 0) issue_S(t, kuse % C::kKS);
+        mma_commit(b_k_empty(kuse % C::kKS));
+        ++kuse;
+        bool started[2] = {false, false};
+        for (int j = 0; alive && j < it.Tmax; ++j) {
+          bool v_used = false, k_next = false;
+          for (int t = 0; t < 2; ++t) {
+            if (j >= T[t]) continue;
+            if (!mbar_wait(b_p_full(t), pc[t] & 1, abort_flag, wait_limit_ns)) {
+              pp_give_up(misc, status, 7);
+              alive = false;
+              break;
+            }
+            ++pc[t];
+            tc_fence_after();
+            const int keep = vdec[t * kDR + (dc[t] % kDR)];
+            ++dc[t];
+            if (keep) {
+              if (!v_used) {
+                if (!mbar_wait(b_v_full(vuse % C::kVS), (vuse / C::kVS) & 1, abort_flag,
+                               wait_limit_ns)) {
+                  pp_give_up(misc, status, 8);
+                  alive = false;
+                  break;
+                }
+                tc_fence_after();
+                v_used = true;
+              }
+              const uint32_t vb = sV + (vuse % C::kVS) * C::kKVBytes;
+#pragma unroll
+              for (int kk = 0; kk < BC / 16; ++kk) {
+                const uint64_t db = sw128_desc(vb + kk * 16 * 128, C::kKVPanel, 1024);
+                mma_ts(tO(t), tS(t) + kk * 8, db, idPV, (started[t] || kk > 0) ? 1u : 0u);
+              }
+              started[t] = true;
+            }
+            if (j == T[t] - 1) mma_commit(b_o_full(t));
+            if (j + 1 < T[t]) {
+              if (!k_next) {
+                if (!mbar_wait(b_k_full(kuse % C::kKS), (kuse / C::kKS) & 1, abort_flag,
+                               wait_limit_ns)) {
+                  pp_give_up(misc, status, 9);
+                  alive = false;
+                  break;
+                }
+                tc_fence_after();
+                k_next = true;
+              }
+              issue_S(t, kuse % C::kKS);
+            }
+          }
+          if (k_next) {
+            mma_commit(b_k_empty(kuse % C::kKS));
+            ++kuse;
+          }
+          if (v_used) {
+            mma_commit(b_v_empty(vuse % C::kVS));
+            ++vuse;
+          }
+        }
+        mma_commit(b_q_empty);
+      }
+      // all issued MMAs must finish before TMEM is released
+      mma_commit(b_q_empty);
+      mbar_drain(b_q_empty, items & 1, wait_limit_ns);
+    }
+  } else {
+    reg_inc<kSoftmaxRegs>();
+    // -------------------------------------------------------- softmax warpgroups
+    const int t = (warp - 4) >> 2;    // row block of the pair
+    const int sw = warp & 3;          // TMEM sub-partition of this warp
+    const int row = sw * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(sw * 32) << 16;
+    const float NEG_INF = -__int_as_float(0x7f800000);
+    int sc = 0, dcount = 0, oc = 0;
+    bool ok = true, failed = false;
+    for (long long idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
+      const Item it = make_item<BC, CAUSAL>(idx, BH, n_pairs, n_rb, N);
+      const int T = t == 0 ? it.T0 : it.T1;
+      if (T == 0) continue;  // this row block does not exist
+      const int rb = it.rb0 + t;
+      const int q_idx = rb * kRows + row;
+      const bool row_valid = q_idx < N;
+      const size_t mask_base =
+          skip_mask ? ((static_cast<size_t>(it.bh) * n_rb + rb) * n_tiles) : 0;
+      float m_exact = NEG_INF, m_ref = NEG_INF, l_sum = 0.f;
+      for (int j = 0; j < T; ++j) {
+        bool waited = !failed && __all_sync(0xffffffffu, mbar_wait(b_s_full(t), sc & 1, abort_flag,
+                                                                     wait_limit_ns));
+        ++sc;
+        // raw scores stay in registers as fp32 bit patterns; the log2 scale is
+        // folded into the max (positive scale) and into the exp FFMA below
+        uint32_t u[BC];
+        float mt = NEG_INF;
+        if (waited) {
+          tc_fence_after();
+          tmem_ld_row<BC>(tS(t) + lane_off, u);
+          tmem_wait_ld();
+          // last visible column of this row in tile j (-1: none); one integer
+          // limit keeps the masking to a compare-select per column
+          const int key0 = j * BC;
+          int lim = min(BC - 1, N - 1 - key0);
+          if (CAUSAL) lim = min(lim, q_idx - key0);
+          if (!row_valid) lim = -1;
+          if (lim < BC - 1) {
+#pragma unroll
+            for (int c = 0; c < BC; ++c) u[c] = (c > lim) ? 0xff800000u : u[c];
+          }
+#pragma unroll
+          for (int c = 0; c < BC; ++c) mt = fmaxf(mt, __uint_as_float(u[c]));
+          mt *= scale_log2;  // log2 units; -inf stays -inf
+        }
+        // ---- skip test: every row of this row block must have mt < m - tau
+        bool skip = false;
+        if (!tau_is_inf) {
+          const bool pass =
+              !row_valid || (m_exact != NEG_INF && (mt == NEG_INF || mt < m_exact - tau_log2));
+          const unsigned all_pass = __all_sync(0xffffffffu, pass);
+          const unsigned all_ok = __all_sync(0xffffffffu, waited);
+          const int slot = j & 1;
+          if (lane == 0)
+            reinterpret_cast<volatile int*>(misc->vote[t][slot])[sw] =
+                (all_pass ? 1 : 0) | (all_ok ? 0 : 2);
+          named_bar(1 + t, 128);
+          int v = 1, bad = 0;
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+            const int vw = reinterpret_cast<volatile int*>(misc->vote[t][slot])[w];
+            v &= vw & 1;
+            bad |= vw & 2;
+          }
+          skip = v != 0;
+          if (bad) waited = false;
+        }
+        if (!waited) {
+          pp_give_up(misc, status, 10);
+          ok = false;
+          break;
+        }
+        m_exact = fmaxf(m_exact, mt);
+        const int di = dcount % kDR;
+        ++dcount;
+        if (row == 0) {
+          vdec[t * kDR + di] = skip ? 0 : 1;
+          if (skip_mask) skip_mask[mask_base + j] = skip ? 1 : 0;
+          mbar_arrive(b_dec(t, di));
+        }
+        if (skip) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(b_p_full(t));
+          continue;
+        }
+        // ---- kept tile: lazy reference max, O rescale (O_t is idle here), P
+        const float m_cand = fmaxf(m_ref, mt);
+        const bool moved = row_valid && (m_cand > m_ref + kRescale);
+        float alpha = 1.f;
+        if (moved) {
+          alpha = ex2(m_ref - m_cand);
+          m_ref = m_cand;
+        }
+        float rs = 0.f;
+        const float neg_m = -m_ref;
+#pragma unroll
+        for (int c0 = 0; c0 < BC; c0 += 32) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            float p0 = ex2(fmaf(__uint_as_float(u[c0 + 2 * c]), scale_log2, neg_m));
+            float p1 = ex2(fmaf(__uint_as_float(u[c0 + 2 * c + 1]), scale_log2, neg_m));
+            if (!row_valid) p0 = p1 = 0.f;
+            const uint32_t w = pack_bf16x2(p0, p1);
+            rs += __uint_as_float(w << 16) + __uint_as_float(w & 0xffff0000u);
+            pk[c] = w;
+          }
+          tmem_st16(tS(t) + lane_off + c0 / 2, pk);
+        }
+        l_sum = l_sum * alpha + rs;
+        // O_t is idle (S_t_j done => PV_t_{j-1} done); rescale after the P
+        // store so the scores are no longer live
+        if (j > 0 && __any_sync(0xffffffffu, moved)) {
+          tc_fence_after();
+          const float a = moved ? alpha : 1.f;
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t r[32];
+            tmem_ld32(tO(t) + lane_off + c0, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * a);
+            tmem_st32(tO(t) + lane_off + c0, r);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(b_p_full(t));
+      }
+      if (!ok) break;
+      // ---- epilogue: O / l -> bf16 -> global; unvisited tiles marked 2
+      if (skip_mask)
+        for (int j = T + row; j < n_tiles; j += 128) skip_mask[mask_base + j] = 2;
+      const bool done =
+          __all_sync(0xffffffffu, mbar_wait(b_o_full(t), oc & 1, abort_flag, wait_limit_ns));
+      ++oc;
+      if (!done) {
+        pp_give_up(misc, status, 11);
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const float inv_l = row_valid ? 1.f / l_sum : 0.f;
+      __nv_bfloat16* orow = O + (static_cast<size_t>(it.bh) * N + (row_valid ? q_idx : 0)) * D;
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t r[32];
+        tmem_ld32(tO(t) + lane_off + c0, r);
+        tmem_wait_ld();
+        if (row_valid) {
+          uint32_t w[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            w[c] = pack_bf16x2(__uint_as_float(r[2 * c]) * inv_l, __uint_as_float(r[2 * c + 1]) * inv_l);
+          uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+        }
+      }
+      // O_t may be overwritten by the next item's first P*V only after this
+      // warpgroup signals that item's first P: ordering comes from p_full.
+      tc_fence_before();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// --------------------------------------------------------------------- host
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 pp_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+bool pp_map(CUtensorMap* m, const void* base, int BH, int rows, int D, int box_rows) {
+  auto enc = pp_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(rows) * D * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int BC, bool CAUSAL>
+int pp_launch(const PrefillLaunch& a) {
+  using C = PPCfg<D, BC>;
+  auto kern = prefill_pp_kernel<D, BC, CAUSAL>;
+  static uint64_t ready = 0;  // one bit per device: attributes set and checked
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return ATTN_ERR_CUDA;
+  static int sm_count[64];
+  if (!(ready >> dev & 1)) {
+    // The register split (setmaxnreg) assumes exactly kPPRegs registers per
+    // thread at launch; anything else could leave setmaxnreg.inc waiting.
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (fa.numRegs != kPPRegs) return ATTN_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+        cudaSuccess)
+      return ATTN_ERR_CUDA;
+    if (cudaDeviceGetAttribute(&sm_count[dev], cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return ATTN_ERR_CUDA;
+    ready |= uint64_t(1) << dev;
+  }
+  CUtensorMap mq, mk, mv;
+  if (!pp_map(&mq, a.Q, a.B * a.Hq, a.N, D, kRows) || !pp_map(&mk, a.K, a.B * a.Hkv, a.N, D, BC) ||
+      !pp_map(&mv, a.V, a.B * a.Hkv, a.N, D, BC))
+    return ATTN_ERR_CUDA;
+  const long long n_rb = (a.N + kRows - 1) / kRows;
+  const long long n_items = static_cast<long long>(a.B) * a.Hq * ((n_rb + 1) / 2);
+  const int grid = static_cast<int>(n_items < sm_count[dev] ? n_items : sm_count[dev]);
+  kern<<<grid, kPPThreads, C::kSmemBytes, a.stream>>>(
+      mq, mk, mv, static_cast<__nv_bfloat16*>(a.O), a.skip_mask, a.status, a.B, a.Hq, a.Hkv, a.N,
+      a.scale_log2, a.tau_log2, a.tau_is_inf, a.wait_limit_ns);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D, int BC>
+int pp_launch_c(const PrefillLaunch& a) {
+  return a.causal ? pp_launch<D, BC, true>(a) : pp_launch<D, BC, false>(a);
+}
+
+}  // namespace
+
+int launch_prefill_pp(const PrefillLaunch& a) {
+  if (a.Br != 128) return ATTN_ERR_INVALID_ARG;
+  if (a.d == 128) return a.Bc == 64 ? pp_launch_c<128, 64>(a) : pp_launch_c<128, 128>(a);
+  if (a.d == 64) return a.Bc == 64 ? pp_launch_c<64, 64>(a) : pp_launch_c<64, 128>(a);
+  return ATTN_ERR_INVALID_ARG;
+}
+
+}  // namespace bss
