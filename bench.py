@@ -281,27 +281,48 @@ def main():
 
         return mor(x, dev)
 
-    def timed(fn, steps, warmup):
+    attempts_log = []
+
+    def timed(fn, steps, warmup, label="step"):
+        """Exactly `steps` calls between two events on the launching stream.
+
+        Per-call events inside the region separate GPU time from host gaps
+        (time the GPU sat idle because the host had not launched yet).  If
+        the host gaps exceed 2% of the region, the region is measured again
+        (at most 3 attempts); every attempt is reported in `timing_attempts`.
+        """
         for _ in range(warmup):
             fn()
-        gc.collect()
-        gc.disable()  # no collector pauses between the two events
-        barrier()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        t0 = time.time()
-        e0.record(stream)
-        for _ in range(steps):
-            fn()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        t1 = time.time()
-        gc.enable()
-        barrier()
-        st = bss.attn_sync_status()
-        if st != 0:
-            raise RuntimeError(f"kernel status {bss.attn_status_string(st)}")
-        return max_over_ranks(e0.elapsed_time(e1) / steps), t0, t1
+        tries = []
+        for attempt in range(3):
+            gc.collect()
+            gc.disable()  # no collector pauses between the two events
+            barrier()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            marks = [torch.cuda.Event(enable_timing=True) for _ in range(2 * steps)]
+            t0 = time.time()
+            e0.record(stream)
+            for i in range(steps):
+                marks[2 * i].record(stream)
+                fn()
+                marks[2 * i + 1].record(stream)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            t1 = time.time()
+            gc.enable()
+            barrier()
+            st = bss.attn_sync_status()
+            if st != 0:
+                raise RuntimeError(f"kernel status {bss.attn_status_string(st)}")
+            total = e0.elapsed_time(e1)
+            busy = sum(marks[2 * i].elapsed_time(marks[2 * i + 1]) for i in range(steps))
+            gap = max(0.0, total - busy)
+            tries.append({"ms_total": total, "host_gap_ms": gap})
+            if gap <= 0.02 * total:
+                break
+        attempts_log.append({"region": label, "attempts": tries})
+        return max_over_ranks(total / steps), t0, t1
 
     vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
     clocks = ClockSampler(int(vis[local]) if local < len(vis) and vis[local].strip().isdigit() else local)
@@ -317,7 +338,7 @@ def main():
     def step():
         bss.prefill(Q, K, V, w["causal"], math.inf, w["Br"], w["Bc"], out=O)
 
-    ms, t0, t1 = timed(step, args.steps, args.warmup)
+    ms, t0, t1 = timed(step, args.steps, args.warmup, "prefill " + MAIN)
     flops = dense_flops(w)
     value = world * flops / (ms * 1e-3) / 1e12
     achieved = flops / (ms * 1e-3) / 1e12
@@ -342,7 +363,7 @@ def main():
         Op.copy_(O, non_blocking=True)
 
     e2e_steps = max(3, min(args.steps, 20))
-    ms_e2e, _, _ = timed(e2e_step, e2e_steps, 2)
+    ms_e2e, _, _ = timed(e2e_step, e2e_steps, 2, "e2e")
     e2e = {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
            "h2d_bytes_per_step": Qp.numel() * 2 + Kp.numel() * 2 + Vp.numel() * 2,
            "d2h_bytes_per_step": Op.numel() * 2, "ms_per_step": ms_e2e,
@@ -355,7 +376,7 @@ def main():
     def prefill_extra(name, wl, Qd, Kd, Vd, tau, steps, warmup):
         Od = torch.empty_like(Qd)
         ms_x, _, _ = timed(lambda: bss.prefill(Qd, Kd, Vd, wl["causal"], tau, wl["Br"], wl["Bc"], out=Od),
-                           steps, warmup)
+                           steps, warmup, f"{name}@tau={tau}")
         _, mask = bss.prefill(Qd, Kd, Vd, wl["causal"], tau, wl["Br"], wl["Bc"], out=Od, skip_mask=True)
         mk = mask[mask != 2]
         f = dense_flops(wl)
@@ -383,7 +404,8 @@ def main():
     decode = {}
     kv_bytes = wd["B"] * wd["Hkv"] * wd["L"] * wd["d"] * 2
     for tau in wd["taus"]:
-        ms_d, d0, d1 = timed(lambda: bss.decode(q, Kd, Vd, tau, out=o), args.steps, args.warmup)
+        ms_d, d0, d1 = timed(lambda: bss.decode(q, Kd, Vd, tau, out=o), args.steps, args.warmup,
+                             f"decode@tau={tau}")
         _, mask = bss.decode(q, Kd, Vd, tau, out=o, skip_mask=True)
         kept = 1.0 - float((mask == 1).float().mean().item())
         read = kv_bytes * (1.0 + kept)
@@ -436,6 +458,7 @@ def main():
             "e2e": e2e, "gpu_launches": args.steps, "clocks": clk, "cpu_baseline": cpu_base,
             "decode": {"metric": "decode KV-read GB/s", "workload": DECODE, **decode},
             "workloads": extras,
+            "timing_attempts": attempts_log,
         }
         print(json.dumps(line), flush=True)
     if dist:

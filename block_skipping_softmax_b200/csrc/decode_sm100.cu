@@ -15,10 +15,15 @@
 // memory ring, issued three tiles ahead; a V tile is requested only once the
 // tile is known to be kept, and consumed two iterations later so its latency
 // stays hidden.  Shared memory is read with 16-byte vector loads, each warp
-// instruction covering whole key rows (conflict-free); dot products use fp32
-// FMAs and a transposing butterfly reduction across the lanes of one key.
-// Output per split: normalised partial o (fp32) and its log2-sum-exp; a
-// second kernel merges the splits exactly.
+// instruction covering whole key rows; dot products use packed fp32 FMAs and
+// a transposing butterfly reduction across the lanes of one key.
+//
+// One CTA barrier per tile: the scores of tile i and each warp's per-row
+// maxima are formed before it; after it every thread takes the same skip
+// decision from the eight warp maxima (no serial phase), the lanes that hold
+// scores turn them into probabilities for a later P*V, and thread 0 refills
+// the copy rings.  Output per split: normalised partial o (fp32) and its
+// log2-sum-exp; a second kernel merges the splits exactly.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -34,38 +39,30 @@ namespace {
 
 constexpr int kWarps = 8;
 constexpr int kDecThreads = kWarps * 32;
-constexpr int kKStages = 3;   // K tiles in flight ahead of the compute
-constexpr int kLag = 2;       // a kept tile's P*V runs kLag iterations after its test
+constexpr int kKStages = 3;  // K tiles in flight ahead of the compute
+constexpr int kLag = 2;      // a kept tile's P*V runs kLag iterations after its test
 constexpr int kVStages = kLag + 1;
-constexpr int kSRing = kLag + 1;
-constexpr int kDRing = 4;
+constexpr int kPRing = kLag + 1;
 
 template <int D, int G>
 struct DecCfg {
   static constexpr int kTileBytes = kDecodeTile * D * 2;
-  static constexpr int kCPK = D / 8;          // 16-byte chunks per key row
-  static constexpr int kKPI = 32 / kCPK;      // keys per warp instruction
-  static constexpr int kIters = (kDecodeTile / kWarps) / kKPI;
+  static constexpr int kCPK = D / 8;                  // 16-byte chunks per key row
+  static constexpr int kKPI = 32 / kCPK;              // keys per warp instruction
+  static constexpr int kKeysPerWarp = kDecodeTile / kWarps;
+  static constexpr int kIters = kKeysPerWarp / kKPI;
+  static constexpr int kLanesPerRow = kCPK / G;       // lanes holding copies of one score
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kOffK + kKStages * kTileBytes;
-  static constexpr int kOffS = kOffV + kVStages * kTileBytes;             // float [SR][G][64]
-  static constexpr int kOffP = kOffS + kSRing * G * kDecodeTile * 4;      // float [64][G]
-  static constexpr int kOffM = kOffP + kDecodeTile * G * 4;               // float [G]
-  static constexpr int kOffDec = kOffM + 64;                              // int [kDRing]
-  static constexpr int kOffBar = kOffDec + 64;                            // k_full, v_full
+  static constexpr int kOffP = kOffV + kVStages * kTileBytes;             // float [PR][64][G]
+  static constexpr int kOffW = kOffP + kPRing * kDecodeTile * G * 4;      // float [2][warps][G]
+  static constexpr int kOffMisc = kOffW + 2 * kWarps * G * 4;
+  static constexpr int kOffBar = kOffMisc + 64;                           // k_full, v_full
   static constexpr int kSmemBytes = kOffBar + 8 * (kKStages + kVStages) + 128;
   // the final cross-warp reduction reuses the K ring
   static_assert(kWarps * G * (D + 1) * 4 <= kKStages * kTileBytes, "reduction scratch");
+  static_assert(G <= kCPK, "rows per group");
 };
-
-__device__ __forceinline__ void bf16x8_to_f32(const uint4& u, float (&f)[8]) {
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    f[2 * i] = __uint_as_float(w[i] << 16);
-    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-  }
-}
 
 }  // namespace
 
@@ -80,13 +77,11 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
   using C = DecCfg<D, G>;
   extern __shared__ __align__(128) uint8_t smem[];
   const uint32_t sbase = smem_u32(smem);
-  float* s_ring = reinterpret_cast<float*>(smem + C::kOffS);
-  float* p_sm = reinterpret_cast<float*>(smem + C::kOffP);
-  float* m_sm = reinterpret_cast<float*>(smem + C::kOffM);
-  volatile int* dec = reinterpret_cast<volatile int*>(smem + C::kOffDec);
-  // Give-ups in this kernel are made CTA-uniform with __syncthreads_or, so no
-  // role ever needs to be told to stop early: the flag stays 0.
-  volatile int* never = reinterpret_cast<volatile int*>(smem + C::kOffDec + 32);
+  float* p_ring = reinterpret_cast<float*>(smem + C::kOffP);
+  float* wmax = reinterpret_cast<float*>(smem + C::kOffW);
+  // Give-ups are made CTA-uniform with __syncthreads_or, so no role ever
+  // needs to be told to stop early: this flag stays 0.
+  volatile int* never = reinterpret_cast<volatile int*>(smem + C::kOffMisc);
   const uint32_t bar0 = sbase + C::kOffBar;
   auto b_k_full = [&](int s) { return bar0 + 8u * s; };
   auto b_v_full = [&](int s) { return bar0 + 8u * (kKStages + s); };
@@ -133,67 +128,77 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
   // this lane's slice: 16-byte chunk `c` of key `sub` within each warp instruction
   const int c = lane % C::kCPK;
   const int sub = lane / C::kCPK;
-  float qf[G][8];
+  const int my_row = c / C::kLanesPerRow;  // the score row this lane ends up holding
+  const bool writer = (c % C::kLanesPerRow) == 0;
+  float2 qf[G][4];
 #pragma unroll
   for (int r = 0; r < G; ++r) {
     const uint4 u = *reinterpret_cast<const uint4*>(
         q + (static_cast<size_t>(b) * Hq + kv * G + r) * D + c * 8);
-    bf16x8_to_f32(u, qf[r]);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+      qf[r][e] = make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xffff0000u));
   }
-  float acc[G][8];
+  float2 acc[G][4];
   float lsum[G];
-  float m_used[G];
+  // every thread keeps identical copies of the decision state
+  float m_exact[G];           // exact running max after the latest tested tile (log2 units)
+  float m_hist[kLag + 1][G];  // m_hist[k][r] = running max after tile i - k
+  float m_acc[G];             // reference max of the partial sums acc / lsum
 #pragma unroll
   for (int r = 0; r < G; ++r) {
     lsum[r] = 0.f;
-    m_used[r] = NEG_INF;
+    m_exact[r] = NEG_INF;
+    m_acc[r] = NEG_INF;
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[r][e] = 0.f;
+    for (int e = 0; e < 4; ++e) acc[r][e] = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int k = 0; k <= kLag; ++k) m_hist[k][r] = NEG_INF;
   }
-  float m_exact[G];  // exact running max of each row (warp 0 keeps it)
-#pragma unroll
-  for (int r = 0; r < G; ++r) m_exact[r] = NEG_INF;
-  int kept_issue = 0;  // V tiles requested (thread 0)
-  int pv_count = 0;    // V tiles consumed
-  bool ok = true;
-  int k_consumed = 0;
+  uint32_t kept_bits = 0;  // bit k: tile i - k was kept
+  int pv_count = 0;        // V tiles consumed
+  bool ok = true;          // this thread's waits so far succeeded
 
   for (int i = 0; i < nt + kLag; ++i) {
-    // ---------------- scores of tile i: s = q . k (log2 units) into the ring
+    // ---------------- A: scores of tile i and the per-warp row maxima
+    float sv[C::kIters];
     if (i < nt) {
       const int ks = i % kKStages;
-      ok = mbar_wait(b_k_full(ks), (i / kKStages) & 1, never, wait_limit_ns);
-    }
-    if (__syncthreads_or(!ok)) {  // uniform give-up
-      ok = false;
-      break;
-    }
-    if (i < nt) {
-      const int ks = i % kKStages;
+      const bool got = mbar_wait(b_k_full(ks), (i / kKStages) & 1, never, wait_limit_ns);
+      ok = ok && got;
       const uint8_t* kt = smem + C::kOffK + ks * C::kTileBytes;
-      float* srow = s_ring + (i % kSRing) * G * kDecodeTile;
       const int key_lim = L - (t_begin + i) * kDecodeTile;  // keys >= key_lim are past L
+      float wm = NEG_INF;
 #pragma unroll
       for (int it = 0; it < C::kIters; ++it) {
-        const int key = warp * (kDecodeTile / kWarps) + it * C::kKPI + sub;
-        const uint4 u = *reinterpret_cast<const uint4*>(kt + key * D * 2 + c * 16);
-        float kf[8];
-        bf16x8_to_f32(u, kf);
+        const int key = warp * C::kKeysPerWarp + it * C::kKPI + sub;
         float v[G];
+        if (got) {
+          const uint4 u = *reinterpret_cast<const uint4*>(kt + key * D * 2 + c * 16);
+          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+          float2 kf[4];
 #pragma unroll
-        for (int r = 0; r < G; ++r) {
-          float sacc = 0.f;
+          for (int e = 0; e < 4; ++e)
+            kf[e] = make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xffff0000u));
 #pragma unroll
-          for (int e = 0; e < 8; ++e) sacc = fmaf(qf[r][e], kf[e], sacc);
-          v[r] = sacc;
+          for (int r = 0; r < G; ++r) {
+            float2 s2 = __fmul2_rn(qf[r][0], kf[0]);
+#pragma unroll
+            for (int e = 1; e < 4; ++e) s2 = __ffma2_rn(qf[r][e], kf[e], s2);
+            v[r] = s2.x + s2.y;
+          }
+        } else {
+#pragma unroll
+          for (int r = 0; r < G; ++r) v[r] = 0.f;
         }
         // transposing butterfly over the kCPK lanes of this key: each halving
         // step keeps half of the rows, so after log2(G) steps a lane owns one
-        // row (row = c / (kCPK/G)); the remaining steps are plain sums
+        // row (my_row); the remaining steps are plain sums
 #pragma unroll
         for (int step = 0; (C::kCPK >> (step + 1)) >= 1; ++step) {
-          const int o = C::kCPK >> (step + 1);  // xor distance of this step
-          const int n = G >> step;               // rows this lane still holds (if >= 1)
+          const int o = C::kCPK >> (step + 1);
+          const int n = G >> step;
           if (n > 1) {
             const int hh = n / 2;
             const bool upper = (lane & o) != 0;
@@ -207,45 +212,44 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
             v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
           }
         }
-        constexpr int kLanesPerRow = C::kCPK / G;
-        if ((c % kLanesPerRow) == 0) {
-          const int r = c / kLanesPerRow;
-          srow[r * kDecodeTile + key] = key < key_lim ? v[0] * scale_log2 : NEG_INF;
-        }
+        sv[it] = key < key_lim ? v[0] * scale_log2 : NEG_INF;
+        wm = fmaxf(wm, sv[it]);
       }
-      ++k_consumed;
+      // max over this warp's keys for my_row: combine the `sub` lanes
+#pragma unroll
+      for (int o = C::kCPK; o < 32; o <<= 1) wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, o));
+      if (writer && sub == 0) wmax[((i & 1) * kWarps + warp) * G + my_row] = wm;
     }
-    __syncthreads();  // S1: scores visible, K slot free
-    // ---------------- skip test for tile i (warp 0), then refill the rings
-    if (warp == 0 && i < nt) {
-      const float* srow = s_ring + (i % kSRing) * G * kDecodeTile;
+    if (__syncthreads_or(!ok)) {  // the single per-tile barrier; also a uniform give-up
+      ok = false;
+      break;
+    }
+    // ---------------- B: decision for tile i (the same in every thread)
+    bool keep_i = false;
+    if (i < nt) {
       bool all_pass = !tau_is_inf;
 #pragma unroll
       for (int r = 0; r < G; ++r) {
-        float mt = fmaxf(srow[r * kDecodeTile + lane], srow[r * kDecodeTile + lane + 32]);
+        float mt = NEG_INF;
 #pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, o));
+        for (int w = 0; w < kWarps; ++w) mt = fmaxf(mt, wmax[((i & 1) * kWarps + w) * G + r]);
         const bool pass = m_exact[r] != NEG_INF && (mt == NEG_INF || mt < m_exact[r] - tau_log2);
         all_pass = all_pass && pass;
         m_exact[r] = fmaxf(m_exact[r], mt);
       }
-      const bool skip = all_pass;
-      if (lane == 0) {
-#pragma unroll
-        for (int r = 0; r < G; ++r) m_sm[r] = m_exact[r];
-        dec[i % kDRing] = skip ? 0 : 1;
-        if (skip_mask)
-          skip_mask[(static_cast<size_t>(b) * Hkv + kv) * n_tiles_all + t_begin + i] = skip ? 1 : 0;
+      keep_i = !all_pass;
+      if (tid == 0) {
         const int t = t_begin + i;
-        if (!skip) {
-          const int vs = kept_issue % kVStages;
+        if (skip_mask)
+          skip_mask[(static_cast<size_t>(b) * Hkv + kv) * n_tiles_all + t] = keep_i ? 0 : 1;
+        if (keep_i) {  // the slot's previous tile finished its P*V before this barrier
+          const int vs = v_issued % kVStages;
           mbar_arrive_expect_tx(b_v_full(vs), tile_bytes(t));
           bulk_load(sbase + C::kOffV + vs * C::kTileBytes,
                     Vg + static_cast<size_t>(t) * kDecodeTile * D, tile_bytes(t), b_v_full(vs));
-          ++kept_issue;
           ++v_issued;
         }
-        if (i + kKStages < nt) {
+        if (i + kKStages < nt) {  // every thread has finished reading K slot i % kKStages
           const int ks = i % kKStages;
           const int tn = t + kKStages;
           mbar_arrive_expect_tx(b_k_full(ks), tile_bytes(tn));
@@ -254,56 +258,70 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
           ++k_issued;
         }
       }
-    }
-    __syncthreads();  // S2: decision and running max visible
-    // ---------------- probabilities of tile t = i - kLag (if kept)
-    const int t = i - kLag;
-    const bool do_pv = (t >= 0) && dec[t % kDRing] != 0;
-    if (do_pv) {
-      const float* srow = s_ring + (t % kSRing) * G * kDecodeTile;
-      for (int idx = tid; idx < G * kDecodeTile; idx += kDecThreads) {
-        const int key = idx / G, r = idx % G;
-        p_sm[idx] = ex2(srow[r * kDecodeTile + key] - m_sm[r]);
-      }
-    }
-    // S3 (uniform): probabilities visible; also carries the V-wait give-up
-    bool vok = true;
-    if (do_pv)
-      vok = mbar_wait(b_v_full(pv_count % kVStages), (pv_count / kVStages) & 1,
-                      never, wait_limit_ns);
-    if (__syncthreads_or(!vok)) {
-      ok = false;
-      break;
-    }
-    if (do_pv) {
-      // move the reference max of this thread's partial sums if it changed
+      // probabilities of tile i relative to the running max after tile i
+      if (keep_i && writer) {
+        float* pr = p_ring + (i % kPRing) * kDecodeTile * G;
+        float mr = NEG_INF;
 #pragma unroll
-      for (int r = 0; r < G; ++r) {
-        const float mn = m_sm[r];
-        if (mn != m_used[r]) {
-          const float a = ex2(m_used[r] - mn);
-          lsum[r] *= a;
+        for (int r = 0; r < G; ++r)
+          if (r == my_row) mr = m_exact[r];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) acc[r][e] *= a;
-          m_used[r] = mn;
+        for (int it = 0; it < C::kIters; ++it) {
+          const int key = warp * C::kKeysPerWarp + it * C::kKPI + sub;
+          pr[key * G + my_row] = ex2(sv[it] - mr);
         }
       }
-      const uint8_t* vt = smem + C::kOffV + (pv_count % kVStages) * C::kTileBytes;
-      const int key_lim = L - (t_begin + t) * kDecodeTile;
+    }
+    // shift the per-tile history: running max after tile i, kept bit of tile i
 #pragma unroll
-      for (int it = 0; it < C::kIters; ++it) {
-        const int key = warp * (kDecodeTile / kWarps) + it * C::kKPI + sub;
-        if (key < key_lim) {
-          float vf[8];
-          bf16x8_to_f32(*reinterpret_cast<const uint4*>(vt + key * D * 2 + c * 16), vf);
-          float p[G];
+    for (int k = kLag; k >= 1; --k)
 #pragma unroll
-          for (int r = 0; r < G; ++r) p[r] = p_sm[key * G + r];
+      for (int r = 0; r < G; ++r) m_hist[k][r] = m_hist[k - 1][r];
 #pragma unroll
-          for (int r = 0; r < G; ++r) {
+    for (int r = 0; r < G; ++r) m_hist[0][r] = m_exact[r];
+    kept_bits = (kept_bits << 1) | (keep_i ? 1u : 0u);
+
+    // ---------------- C: P*V of tile t = i - kLag (its p were written kLag barriers ago)
+    const int t = i - kLag;
+    if (t >= 0 && ((kept_bits >> kLag) & 1u)) {
+      const int vs = pv_count % kVStages;
+      const bool got = mbar_wait(b_v_full(vs), (pv_count / kVStages) & 1, never, wait_limit_ns);
+      ok = ok && got;  // acted on at the next barrier
+      if (got) {
+        // move the reference max of the partial sums up to this tile's
 #pragma unroll
-            for (int e = 0; e < 8; ++e) acc[r][e] = fmaf(p[r], vf[e], acc[r][e]);
-            if (c == 0) lsum[r] += p[r];
+        for (int r = 0; r < G; ++r) {
+          const float mn = m_hist[kLag][r];
+          if (mn != m_acc[r]) {
+            const float a = ex2(m_acc[r] - mn);  // m_acc = -inf initially gives 0
+            lsum[r] *= a;
+            const float2 a2 = make_float2(a, a);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[r][e] = __fmul2_rn(acc[r][e], a2);
+            m_acc[r] = mn;
+          }
+        }
+        const uint8_t* vt = smem + C::kOffV + vs * C::kTileBytes;
+        const float* pr = p_ring + (t % kPRing) * kDecodeTile * G;
+        const int key_lim = L - (t_begin + t) * kDecodeTile;
+#pragma unroll
+        for (int it = 0; it < C::kIters; ++it) {
+          const int key = warp * C::kKeysPerWarp + it * C::kKPI + sub;
+          if (key < key_lim) {
+            const uint4 u = *reinterpret_cast<const uint4*>(vt + key * D * 2 + c * 16);
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+            float2 vf[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              vf[e] = make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xffff0000u));
+#pragma unroll
+            for (int r = 0; r < G; ++r) {
+              const float pv = pr[key * G + r];
+              const float2 p2 = make_float2(pv, pv);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) acc[r][e] = __ffma2_rn(p2, vf[e], acc[r][e]);
+              if (c == 0) lsum[r] += pv;
+            }
           }
         }
       }
@@ -311,13 +329,16 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
     }
   }
 
-  if (!ok) {
-    // leave no bulk copy in flight into this CTA's shared memory
+  // a V wait in the last iterations may have failed after the last barrier
+  if (__syncthreads_or(!ok)) {
+    // leave no bulk copy in flight into this CTA's shared memory: the last
+    // copy issued into each ring slot is waited for (earlier ones in the same
+    // slot completed before it was reused)
     if (tid == 0) {
       atomicCAS(status, 0, ATTN_DEVICE_TIMEOUT_BASE + 20);
-      for (int k = k_consumed; k < k_issued; ++k)
+      for (int k = max(0, k_issued - kKStages); k < k_issued; ++k)
         mbar_drain(b_k_full(k % kKStages), (k / kKStages) & 1, wait_limit_ns);
-      for (int k = pv_count; k < v_issued; ++k)
+      for (int k = max(0, v_issued - kVStages); k < v_issued; ++k)
         mbar_drain(b_v_full(k % kVStages), (k / kVStages) & 1, wait_limit_ns);
     }
     return;
@@ -330,7 +351,10 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
     for (int r = 0; r < G; ++r) {
       lsum[r] += __shfl_xor_sync(0xffffffffu, lsum[r], o);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[r][e] += __shfl_xor_sync(0xffffffffu, acc[r][e], o);
+      for (int e = 0; e < 4; ++e) {
+        acc[r][e].x += __shfl_xor_sync(0xffffffffu, acc[r][e].x, o);
+        acc[r][e].y += __shfl_xor_sync(0xffffffffu, acc[r][e].y, o);
+      }
     }
   }
   float* red = reinterpret_cast<float*>(smem + C::kOffK);  // [warp][G][D+1]
@@ -339,7 +363,10 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
 #pragma unroll
     for (int r = 0; r < G; ++r) {
 #pragma unroll
-      for (int e = 0; e < 8; ++e) red[(warp * G + r) * (D + 1) + c * 8 + e] = acc[r][e];
+      for (int e = 0; e < 4; ++e) {
+        red[(warp * G + r) * (D + 1) + c * 8 + 2 * e] = acc[r][e].x;
+        red[(warp * G + r) * (D + 1) + c * 8 + 2 * e + 1] = acc[r][e].y;
+      }
       if (c == 0) red[(warp * G + r) * (D + 1) + D] = lsum[r];
     }
   }
@@ -349,17 +376,24 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
     float s = 0.f;
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) s += red[(w * G + r) * (D + 1) + col];
-    red[(0 * G + r) * (D + 1) + col] = s;  // warp-0 slot is read below only after the sync
+    red[r * (D + 1) + col] = s;  // warp 0's slot; only this thread touches (r, col)
   }
   __syncthreads();
   for (int idx = tid; idx < G * D; idx += kDecThreads) {
     const int r = idx / D, col = idx % D;
-    const float l = red[r * (D + 1) + D];
     const size_t row = static_cast<size_t>(b) * Hq + kv * G + r;
-    o_part[(row * n_splits + split) * D + col] = red[r * (D + 1) + col] / l;
-    // m_sm holds the reference max of the partial sums: skipped tiles never
-    // move the running max, so it equals the value used by the last P*V
-    if (col == 0) lse_part[row * n_splits + split] = m_sm[r] + __log2f(l);
+    o_part[(row * n_splits + split) * D + col] = red[r * (D + 1) + col] / red[r * (D + 1) + D];
+  }
+  if (tid < G) {
+    // every thread holds the same reference max (skipped tiles never move the
+    // running max, so it is the value used by the last P*V); select it with a
+    // constant index
+    float mr = NEG_INF;
+#pragma unroll
+    for (int r = 0; r < G; ++r)
+      if (r == tid) mr = m_acc[r];
+    const size_t row = static_cast<size_t>(b) * Hq + kv * G + tid;
+    lse_part[row * n_splits + split] = mr + __log2f(red[tid * (D + 1) + D]);
   }
 }
 

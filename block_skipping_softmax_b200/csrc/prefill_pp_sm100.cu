@@ -50,13 +50,16 @@ struct PPCfg {
   static constexpr int kKVPanel = BC * 128;
   static constexpr int kKS = (BC == 128 && D == 128) ? 2 : 3;
   static constexpr int kVS = (BC == 128 && D == 128) ? 2 : 3;
-  static constexpr int kOffQ = 0;                                 // two Q tiles
-  static constexpr int kOffK = kOffQ + 2 * kQTile;
+  // Q slots: with two, the next work item's Q loads while this one runs
+  static constexpr int kQS = (BC == 128 && D == 128) ? 1 : 2;
+  static constexpr int kQSlot = 2 * kQTile;                      // two row blocks
+  static constexpr int kOffQ = 0;
+  static constexpr int kOffK = kOffQ + kQS * kQSlot;
   static constexpr int kOffV = kOffK + kKS * kKVBytes;
   static constexpr int kOffBar = kOffV + kVS * kKVBytes;
-  // q_full, q_empty, k_full[KS], k_empty[KS], v_full[VS], v_empty[VS],
-  // s_full[2], p_full[2], o_full[2], dec_full[2][DR]
-  static constexpr int kNumBars = 2 + 2 * kKS + 2 * kVS + 6 + 2 * kDR;
+  // k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[2], p_full[2],
+  // o_full[2], dec_full[2][DR], q_full[QS], q_empty[QS], mma_done
+  static constexpr int kNumBars = 2 * kKS + 2 * kVS + 6 + 2 * kDR + 2 * kQS + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 256 + 1024;
   static constexpr int kTmemCols = 512;
@@ -136,16 +139,19 @@ __global__ void __launch_bounds__(kPPThreads, 1)
   const uint32_t sK = sbase + C::kOffK;
   const uint32_t sV = sbase + C::kOffV;
   const uint32_t bar0 = sbase + C::kOffBar;
-  const uint32_t b_q_full = bar0, b_q_empty = bar0 + 8;
-  auto b_k_full = [&](int s) { return bar0 + 8u * (2 + s); };
-  auto b_k_empty = [&](int s) { return bar0 + 8u * (2 + C::kKS + s); };
-  auto b_v_full = [&](int s) { return bar0 + 8u * (2 + 2 * C::kKS + s); };
-  auto b_v_empty = [&](int s) { return bar0 + 8u * (2 + 2 * C::kKS + C::kVS + s); };
-  constexpr int kB = 2 + 2 * C::kKS + 2 * C::kVS;
+  auto b_k_full = [&](int s) { return bar0 + 8u * s; };
+  auto b_k_empty = [&](int s) { return bar0 + 8u * (C::kKS + s); };
+  auto b_v_full = [&](int s) { return bar0 + 8u * (2 * C::kKS + s); };
+  auto b_v_empty = [&](int s) { return bar0 + 8u * (2 * C::kKS + C::kVS + s); };
+  constexpr int kB = 2 * C::kKS + 2 * C::kVS;
   auto b_s_full = [&](int t) { return bar0 + 8u * (kB + t); };
   auto b_p_full = [&](int t) { return bar0 + 8u * (kB + 2 + t); };
   auto b_o_full = [&](int t) { return bar0 + 8u * (kB + 4 + t); };
   auto b_dec = [&](int t, int i) { return bar0 + 8u * (kB + 6 + t * kDR + i); };
+  constexpr int kBQ = kB + 6 + 2 * kDR;
+  auto b_q_full = [&](int s) { return bar0 + 8u * (kBQ + s); };
+  auto b_q_empty = [&](int s) { return bar0 + 8u * (kBQ + C::kQS + s); };
+  const uint32_t b_mma_done = bar0 + 8u * (kBQ + 2 * C::kQS);
   PPMisc* misc = reinterpret_cast<PPMisc*>(smem + C::kOffMisc);
   volatile int* abort_flag = &misc->abort;
   volatile int* vdec = &misc->dec[0][0];
@@ -160,8 +166,11 @@ __global__ void __launch_bounds__(kPPThreads, 1)
   const long long n_items = static_cast<long long>(BH) * n_pairs;
 
   if (threadIdx.x == 0) {
-    mbar_init(b_q_full, 1);
-    mbar_init(b_q_empty, 1);
+    for (int s = 0; s < C::kQS; ++s) {
+      mbar_init(b_q_full(s), 1);
+      mbar_init(b_q_empty(s), 1);
+    }
+    mbar_init(b_mma_done, 1);
     for (int s = 0; s < C::kKS; ++s) {
       mbar_init(b_k_full(s), 1);
       mbar_init(b_k_empty(s), 1);
@@ -200,17 +209,18 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       for (long long idx = blockIdx.x; alive && idx < n_items; idx += gridDim.x, ++items) {
         const Item it = make_item<BC, CAUSAL>(idx, BH, n_pairs, n_rb, N);
         const int bkv = (it.bh / Hq) * Hkv + (it.bh % Hq) / g;
-        if (items > 0 &&
-            !mbar_wait(b_q_empty, (items - 1) & 1, abort_flag, wait_limit_ns)) {
+        const int qs = items % C::kQS;
+        if (items >= C::kQS && !mbar_wait(b_q_empty(qs), ((items / C::kQS) - 1) & 1, abort_flag,
+                                          wait_limit_ns)) {
           pp_give_up(misc, status, 1);
           break;
         }
         const int nq = it.T1 > 0 ? 2 : 1;
-        mbar_arrive_expect_tx(b_q_full, nq * C::kQTile);
+        mbar_arrive_expect_tx(b_q_full(qs), nq * C::kQTile);
         for (int t = 0; t < nq; ++t)
           for (int p = 0; p < C::kPanels; ++p)
-            tma_load_3d(sQ + t * C::kQTile + p * C::kQPanel, &tmQ, b_q_full, p * 64,
-                        (it.rb0 + t) * kRows, it.bh);
+            tma_load_3d(sQ + qs * C::kQSlot + t * C::kQTile + p * C::kQPanel, &tmQ, b_q_full(qs),
+                        p * 64, (it.rb0 + t) * kRows, it.bh);
         for (int j = 0; j < it.Tmax; ++j) {
           const int s = kload % C::kKS;
           if (kload >= C::kKS &&
@@ -228,7 +238,8 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         kdone = items + 1;
       }
       // never leave with a copy in flight
-      if (kdone > 0) mbar_drain(b_q_full, (kdone - 1) & 1, wait_limit_ns);
+      for (int i = max(0, kdone - C::kQS); i < kdone; ++i)
+        mbar_drain(b_q_full(i % C::kQS), (i / C::kQS) & 1, wait_limit_ns);
       for (int t = max(0, kload - C::kKS); t < kload; ++t)
         mbar_drain(b_k_full(t % C::kKS), (t / C::kKS) & 1, wait_limit_ns);
     } else if (warp == 2 && lane == 0) {
@@ -291,11 +302,13 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       int kuse = 0, vuse = 0, items = 0;
       int pc[2] = {0, 0}, dc[2] = {0, 0};
       bool alive = true;
+      uint32_t q_base = sQ;
       auto issue_S = [&](int t, int kslot) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk & 3) * 32;
-          const uint64_t da = sw128_desc(sQ + t * C::kQTile + (kk >> 2) * C::kQPanel + off, 16, 1024);
+          const uint64_t da =
+              sw128_desc(q_base + t * C::kQTile + (kk >> 2) * C::kQPanel + off, 16, 1024);
           const uint64_t db =
               sw128_desc(sK + kslot * C::kKVBytes + (kk >> 2) * C::kKVPanel + off, 16, 1024);
           mma_ss(tS(t), da, db, idS, kk > 0 ? 1u : 0u);
@@ -305,7 +318,9 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       for (long long idx = blockIdx.x; alive && idx < n_items; idx += gridDim.x, ++items) {
         const Item it = make_item<BC, CAUSAL>(idx, BH, n_pairs, n_rb, N);
         const int T[2] = {it.T0, it.T1};
-        if (!mbar_wait(b_q_full, items & 1, abort_flag, wait_limit_ns)) {
+        const int qs = items % C::kQS;
+        q_base = sQ + qs * C::kQSlot;
+        if (!mbar_wait(b_q_full(qs), (items / C::kQS) & 1, abort_flag, wait_limit_ns)) {
           pp_give_up(misc, status, 5);
           break;
         }
@@ -319,6 +334,8 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           if (T[t] > 0) issue_S(t, kuse % C::kKS);
         mma_commit(b_k_empty(kuse % C::kKS));
         ++kuse;
+        // the Q slot is free once the item's last S MMA has run
+        if (it.Tmax == 1) mma_commit(b_q_empty(qs));
         bool started[2] = {false, false};
         for (int j = 0; alive && j < it.Tmax; ++j) {
           bool v_used = false, k_next = false;
@@ -371,16 +388,16 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             mma_commit(b_k_empty(kuse % C::kKS));
             ++kuse;
           }
+          if (j + 2 == it.Tmax) mma_commit(b_q_empty(qs));  // S MMAs of tile Tmax-1 issued
           if (v_used) {
             mma_commit(b_v_empty(vuse % C::kVS));
             ++vuse;
           }
         }
-        mma_commit(b_q_empty);
       }
       // all issued MMAs must finish before TMEM is released
-      mma_commit(b_q_empty);
-      mbar_drain(b_q_empty, items & 1, wait_limit_ns);
+      mma_commit(b_mma_done);
+      mbar_drain(b_mma_done, 0, wait_limit_ns);
     }
   } else {
     reg_inc<kSoftmaxRegs>();
