@@ -34,9 +34,10 @@ namespace bss {
 namespace {
 
 constexpr int kPPThreads = 384;
-constexpr int kPPRegs = 168;       // registers per thread at launch (checked on the host)
-constexpr int kProducerRegs = 56;  // 128 x 56 + 256 x 224 = 384 x 168
-constexpr int kSoftmaxRegs = 224;
+constexpr int kPPRegs = 168;  // registers per thread at launch (checked on the host)
+#ifndef PP_BC128_PRODUCER_REGS
+#define PP_BC128_PRODUCER_REGS 72
+#endif
 constexpr int kRows = 128;         // rows per tile (row block)
 constexpr int kDR = 4;             // decision ring
 constexpr float kRescale = 8.0f;   // lazy rescale threshold (log2 units)
@@ -63,6 +64,12 @@ struct PPCfg {
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 256 + 1024;
   static constexpr int kTmemCols = 512;
+  // setmaxnreg split of the 384 x 168 launch registers: 128 producer threads
+  // (TMA, MMA issue) and 256 softmax threads.  At 72 the MMA-issuing thread
+  // does not spill; the 128-column softmax needs the larger share.
+  static constexpr int kProducerRegs = (BC == 64) ? 72 : PP_BC128_PRODUCER_REGS;
+  static constexpr int kSoftmaxRegs = (kPPThreads * kPPRegs - 128 * kProducerRegs) / 256 / 8 * 8;
+  static_assert(128 * kProducerRegs + 256 * kSoftmaxRegs <= kPPThreads * kPPRegs, "register split");
   static_assert(2 * D + 2 * BC <= 512, "TMEM budget");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 };
@@ -201,7 +208,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
   auto tS = [&](int t) { return tmem + 2 * D + t * BC; };
 
   if (warp < 4) {
-    reg_dec<kProducerRegs>();
+    reg_dec<C::kProducerRegs>();
     if (warp == 0 && lane == 0) {
       // ---------------------------------------------------- Q and K producer
       int kload = 0, items = 0, kdone = 0;
@@ -273,7 +280,9 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           // V_j is loaded as soon as either row block keeps tile j; every
           // decision is still consumed, in order
           bool issued = false;
-          for (int t = 0; alive && t < 2; ++t) {
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (!alive) break;
             if (j >= T[t]) continue;
             const int di = dl[t] % kDR;
             if (!mbar_wait(b_dec(t, di), (dl[t] / kDR) & 1, abort_flag, wait_limit_ns)) {
@@ -302,16 +311,20 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       int kuse = 0, vuse = 0, items = 0;
       int pc[2] = {0, 0}, dc[2] = {0, 0};
       bool alive = true;
-      uint32_t q_base = sQ;
+      // Descriptors differ only in their start-address field (bits 0-13, in
+      // 16-byte units), so each MMA adds a compile-time offset to a base.
+      constexpr uint32_t kHi = sw128_desc_hi(1024);
+      const uint32_t dK0 = sw128_desc_lo(sK, 16);
+      const uint32_t dV0 = sw128_desc_lo(sV, C::kKVPanel);
+      uint32_t dQ = sw128_desc_lo(sQ, 16);  // this item's Q slot
       auto issue_S = [&](int t, int kslot) {
+        const uint32_t a0 = dQ + t * (C::kQTile >> 4);
+        const uint32_t b0 = dK0 + kslot * (C::kKVBytes >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk & 3) * 32;
-          const uint64_t da =
-              sw128_desc(q_base + t * C::kQTile + (kk >> 2) * C::kQPanel + off, 16, 1024);
-          const uint64_t db =
-              sw128_desc(sK + kslot * C::kKVBytes + (kk >> 2) * C::kKVPanel + off, 16, 1024);
-          mma_ss(tS(t), da, db, idS, kk > 0 ? 1u : 0u);
+          const uint32_t oq = ((kk >> 2) * C::kQPanel + (kk & 3) * 32) >> 4;
+          const uint32_t ok_ = ((kk >> 2) * C::kKVPanel + (kk & 3) * 32) >> 4;
+          mma_ss(tS(t), desc_join(a0 + oq, kHi), desc_join(b0 + ok_, kHi), idS, kk > 0 ? 1u : 0u);
         }
         mma_commit(b_s_full(t));
       };
@@ -319,7 +332,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         const Item it = make_item<BC, CAUSAL>(idx, BH, n_pairs, n_rb, N);
         const int T[2] = {it.T0, it.T1};
         const int qs = items % C::kQS;
-        q_base = sQ + qs * C::kQSlot;
+        dQ = sw128_desc_lo(sQ + qs * C::kQSlot, 16);
         if (!mbar_wait(b_q_full(qs), (items / C::kQS) & 1, abort_flag, wait_limit_ns)) {
           pp_give_up(misc, status, 5);
           break;
@@ -330,6 +343,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           break;
         }
         tc_fence_after();
+#pragma unroll
         for (int t = 0; t < 2; ++t)
           if (T[t] > 0) issue_S(t, kuse % C::kKS);
         mma_commit(b_k_empty(kuse % C::kKS));
@@ -339,6 +353,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         bool started[2] = {false, false};
         for (int j = 0; alive && j < it.Tmax; ++j) {
           bool v_used = false, k_next = false;
+#pragma unroll
           for (int t = 0; t < 2; ++t) {
             if (j >= T[t]) continue;
             if (!mbar_wait(b_p_full(t), pc[t] & 1, abort_flag, wait_limit_ns)) {
@@ -361,12 +376,11 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                 tc_fence_after();
                 v_used = true;
               }
-              const uint32_t vb = sV + (vuse % C::kVS) * C::kKVBytes;
+              const uint32_t vb = dV0 + (vuse % C::kVS) * (C::kKVBytes >> 4);
 #pragma unroll
-              for (int kk = 0; kk < BC / 16; ++kk) {
-                const uint64_t db = sw128_desc(vb + kk * 16 * 128, C::kKVPanel, 1024);
-                mma_ts(tO(t), tS(t) + kk * 8, db, idPV, (started[t] || kk > 0) ? 1u : 0u);
-              }
+              for (int kk = 0; kk < BC / 16; ++kk)
+                mma_ts(tO(t), tS(t) + kk * 8, desc_join(vb + ((kk * 16 * 128) >> 4), kHi), idPV,
+                       (started[t] || kk > 0) ? 1u : 0u);
               started[t] = true;
             }
             if (j == T[t] - 1) mma_commit(b_o_full(t));
@@ -400,7 +414,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       mbar_drain(b_mma_done, 0, wait_limit_ns);
     }
   } else {
-    reg_inc<kSoftmaxRegs>();
+    reg_inc<C::kSoftmaxRegs>();
     // -------------------------------------------------------- softmax warpgroups
     const int t = (warp - 4) >> 2;    // row block of the pair
     const int sw = warp & 3;          // TMEM sub-partition of this warp
@@ -441,9 +455,14 @@ __global__ void __launch_bounds__(kPPThreads, 1)
 #pragma unroll
             for (int c = 0; c < BC; ++c) u[c] = (c > lim) ? 0xff800000u : u[c];
           }
+          // row max: four independent chains of three-input maxima
+          float m4[4] = {NEG_INF, NEG_INF, NEG_INF, NEG_INF};
 #pragma unroll
-          for (int c = 0; c < BC; ++c) mt = fmaxf(mt, __uint_as_float(u[c]));
-          mt *= scale_log2;  // log2 units; -inf stays -inf
+          for (int c = 0; c < BC; c += 8)
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              m4[k] = fmax3(m4[k], __uint_as_float(u[c + 2 * k]), __uint_as_float(u[c + 2 * k + 1]));
+          mt = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * scale_log2;  // log2 units; -inf stays -inf
         }
         // ---- skip test: every row of this row block must have mt < m - tau
         bool skip = false;
@@ -493,22 +512,27 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           alpha = ex2(m_ref - m_cand);
           m_ref = m_cand;
         }
-        float rs = 0.f;
-        const float neg_m = -m_ref;
+        // P = 2^(s*scale - m_ref): one packed FFMA per pair, two ex2, one
+        // pack; the row sum adds the bf16-rounded pair with one packed add
+        const float neg_m = row_valid ? -m_ref : 0.f;  // invalid rows: all scores -inf -> P = 0
+        const float2 sc2 = make_float2(scale_log2, scale_log2);
+        const float2 nm2 = make_float2(neg_m, neg_m);
+        float2 rs2 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int c0 = 0; c0 < BC; c0 += 32) {
           uint32_t pk[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            float p0 = ex2(fmaf(__uint_as_float(u[c0 + 2 * c]), scale_log2, neg_m));
-            float p1 = ex2(fmaf(__uint_as_float(u[c0 + 2 * c + 1]), scale_log2, neg_m));
-            if (!row_valid) p0 = p1 = 0.f;
-            const uint32_t w = pack_bf16x2(p0, p1);
-            rs += __uint_as_float(w << 16) + __uint_as_float(w & 0xffff0000u);
+            const float2 x = __ffma2_rn(
+                make_float2(__uint_as_float(u[c0 + 2 * c]), __uint_as_float(u[c0 + 2 * c + 1])), sc2,
+                nm2);
+            const uint32_t w = pack_bf16x2(ex2(x.x), ex2(x.y));
+            rs2 = __fadd2_rn(rs2, make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)));
             pk[c] = w;
           }
           tmem_st16(tS(t) + lane_off + c0 / 2, pk);
         }
+        const float rs = rs2.x + rs2.y;
         l_sum = l_sum * alpha + rs;
         // O_t is idle (S_t_j done => PV_t_{j-1} done); rescale after the P
         // store so the scores are no longer live
