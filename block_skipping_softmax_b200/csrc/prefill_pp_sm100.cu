@@ -10,16 +10,25 @@
 // Layout of one CTA (384 threads, one per SM, persistent):
 //   warpgroup 0: warp 0 TMA Q (both tiles) + K ring; warp 1 TMEM allocator
 //                and the single MMA-issuing thread; warp 2 TMA V ring
-//                (gated by the skip decisions); warp 3 idle.  56 registers.
-//   warpgroup 1: softmax of row block 0 (thread r owns row r).  224 registers.
-//   warpgroup 2: softmax of row block 1.                        224 registers.
-// TMEM (512 columns): O0 | O1 | S0 | S1, with P_t (bf16) written over S_t.
-// MMA issue order per key tile j:   PV0_j, S0_{j+1}, PV1_j, S1_{j+1}
-// so the exponentials of one row block overlap the other block's MMAs.  A
-// completed S_t_{j+1} implies PV_t_j completed (one thread issues them in
-// order), so softmax t may rescale O_t in TMEM without any further wait.
-// Every wait is bounded; a wait that gives up records a status code and the
-// CTA unwinds (leaving no copy or MMA in flight and freeing TMEM).
+//                (gated by the skip decisions); warp 3 idle.
+//   warpgroup 1: softmax of row block 0 (thread r owns row r).
+//   warpgroup 2: softmax of row block 1.
+// TMEM (512 columns): O0 | O1 | S/P buffers (two per row block when Bc = 64,
+// one when Bc = 128), P_t (bf16) written over S_t.
+// MMA issue order per key tile j and row block t:  PV_t_j, S_t_{j+SB}, commit
+// so the exponentials of one row block overlap the other block's MMAs.
+//
+// Completion signalling.  A tcgen05.commit stalls the MMA pipe for a few
+// hundred cycles, so the issuer makes exactly one commit per row block and
+// step (plus the first SB S tiles of a work item and one Q-slot release per
+// item), into a ring of mbarriers indexed by a running commit count.  Every
+// completion that a role needs is one of those commits:
+//   S_t of key tile i ready         commit #(base_t + i)
+//   P*V_t of key tile j finished    commit #(base_t + min(SB, T_t) + j)
+// (one thread issues every MMA in order, so a commit covers all earlier
+// MMAs).  K and V ring slots, the O rescale and the epilogue all wait on
+// these.  Every wait is bounded; a wait that gives up records a status code
+// and the CTA unwinds (leaving no copy or MMA in flight and freeing TMEM).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -35,12 +44,10 @@ namespace {
 
 constexpr int kPPThreads = 384;
 constexpr int kPPRegs = 168;  // registers per thread at launch (checked on the host)
-#ifndef PP_BC128_PRODUCER_REGS
-#define PP_BC128_PRODUCER_REGS 72
-#endif
-constexpr int kRows = 128;         // rows per tile (row block)
-constexpr int kDR = 4;             // decision ring
-constexpr float kRescale = 8.0f;   // lazy rescale threshold (log2 units)
+constexpr int kRows = 128;    // rows per tile (row block)
+constexpr int kDR = 4;        // decision ring
+constexpr int kCR = 16;       // commit ring per row block (waiters lag by at most ~6)
+constexpr float kRescale = 8.0f;  // lazy rescale threshold (log2 units)
 
 template <int D, int BC>
 struct PPCfg {
@@ -51,27 +58,30 @@ struct PPCfg {
   static constexpr int kKVPanel = BC * 128;
   static constexpr int kKS = (BC == 128 && D == 128) ? 2 : 3;
   static constexpr int kVS = (BC == 128 && D == 128) ? 2 : 3;
+  // S/P buffers per row block: two when TMEM has room (Bc = 64), so the MMA
+  // for key tile j+1 runs while the softmax works on tile j
+  static constexpr int kSB = (2 * D + 4 * BC <= 512) ? 2 : 1;
   // Q slots: with two, the next work item's Q loads while this one runs
   static constexpr int kQS = (BC == 128 && D == 128) ? 1 : 2;
-  static constexpr int kQSlot = 2 * kQTile;                      // two row blocks
+  static constexpr int kQSlot = 2 * kQTile;  // two row blocks
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQS * kQSlot;
   static constexpr int kOffV = kOffK + kKS * kKVBytes;
   static constexpr int kOffBar = kOffV + kVS * kKVBytes;
-  // k_full[KS], k_empty[KS], v_full[VS], v_empty[VS], s_full[2], p_full[2],
-  // o_full[2], dec_full[2][DR], q_full[QS], q_empty[QS], mma_done
-  static constexpr int kNumBars = 2 * kKS + 2 * kVS + 6 + 2 * kDR + 2 * kQS + 1;
+  // k_full[KS], v_full[VS], commit ring[2][CR], p_full[2][SB], dec[2][DR],
+  // q_full[QS], q_empty[QS], mma_done
+  static constexpr int kNumBars = kKS + kVS + 2 * kCR + 2 * kSB + 2 * kDR + 2 * kQS + 1;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 256 + 1024;
   static constexpr int kTmemCols = 512;
   // setmaxnreg split of the 384 x 168 launch registers: 128 producer threads
-  // (TMA, MMA issue) and 256 softmax threads.  At 72 the MMA-issuing thread
-  // does not spill; the 128-column softmax needs the larger share.
-  static constexpr int kProducerRegs = (BC == 64) ? 72 : PP_BC128_PRODUCER_REGS;
+  // (TMA, MMA issue) and 256 softmax threads; at 72 the MMA issuer does not spill
+  static constexpr int kProducerRegs = 72;
   static constexpr int kSoftmaxRegs = (kPPThreads * kPPRegs - 128 * kProducerRegs) / 256 / 8 * 8;
   static_assert(128 * kProducerRegs + 256 * kSoftmaxRegs <= kPPThreads * kPPRegs, "register split");
-  static_assert(2 * D + 2 * BC <= 512, "TMEM budget");
+  static_assert(2 * D + 2 * kSB * BC <= 512, "TMEM budget");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+  static_assert(kKS + kSB + 1 < kCR && kVS + kSB + 1 < kCR, "commit ring too small");
 };
 
 struct PPMisc {
@@ -128,6 +138,30 @@ __device__ __forceinline__ Item make_item(long long idx, int BH, int n_pairs, in
   return it;
 }
 
+// Commits a row block makes in one work item: its first SB S tiles, then one
+// per key tile it visits.
+template <int SB>
+__device__ __forceinline__ int commits_of(int T) { return T > 0 ? min(SB, T) + T : 0; }
+
+// A short FIFO of ring-slot releases: (row block, commit index) that must
+// complete before the slot's next copy.  Fixed positions keep it in registers.
+// The tile number g (running over work items) says when a wait is not needed.
+struct Pending3 {
+  int r[3], c[3], g[3], n;
+  __device__ __forceinline__ void init() { n = 0; }
+  __device__ __forceinline__ void push(int rr, int cc, int gg) {
+    if (n == 0) { r[0] = rr; c[0] = cc; g[0] = gg; }
+    else if (n == 1) { r[1] = rr; c[1] = cc; g[1] = gg; }
+    else { r[2] = rr; c[2] = cc; g[2] = gg; }
+    ++n;
+  }
+  __device__ __forceinline__ void pop() {
+    r[0] = r[1]; c[0] = c[1]; g[0] = g[1];
+    r[1] = r[2]; c[1] = c[2]; g[1] = g[2];
+    --n;
+  }
+};
+
 }  // namespace
 
 template <int D, int BC, bool CAUSAL>
@@ -138,6 +172,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                       int Hkv, int N, float scale_log2, float tau_log2, int tau_is_inf,
                       unsigned long long wait_limit_ns) {
   using C = PPCfg<D, BC>;
+  constexpr int SB = C::kSB;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -147,21 +182,24 @@ __global__ void __launch_bounds__(kPPThreads, 1)
   const uint32_t sV = sbase + C::kOffV;
   const uint32_t bar0 = sbase + C::kOffBar;
   auto b_k_full = [&](int s) { return bar0 + 8u * s; };
-  auto b_k_empty = [&](int s) { return bar0 + 8u * (C::kKS + s); };
-  auto b_v_full = [&](int s) { return bar0 + 8u * (2 * C::kKS + s); };
-  auto b_v_empty = [&](int s) { return bar0 + 8u * (2 * C::kKS + C::kVS + s); };
-  constexpr int kB = 2 * C::kKS + 2 * C::kVS;
-  auto b_s_full = [&](int t) { return bar0 + 8u * (kB + t); };
-  auto b_p_full = [&](int t) { return bar0 + 8u * (kB + 2 + t); };
-  auto b_o_full = [&](int t) { return bar0 + 8u * (kB + 4 + t); };
-  auto b_dec = [&](int t, int i) { return bar0 + 8u * (kB + 6 + t * kDR + i); };
-  constexpr int kBQ = kB + 6 + 2 * kDR;
+  auto b_v_full = [&](int s) { return bar0 + 8u * (C::kKS + s); };
+  constexpr int kBC = C::kKS + C::kVS;
+  auto b_cm = [&](int t, int i) { return bar0 + 8u * (kBC + t * kCR + (i % kCR)); };
+  constexpr int kBP = kBC + 2 * kCR;
+  auto b_p_full = [&](int t, int b) { return bar0 + 8u * (kBP + t * SB + b); };
+  constexpr int kBD = kBP + 2 * SB;
+  auto b_dec = [&](int t, int i) { return bar0 + 8u * (kBD + t * kDR + i); };
+  constexpr int kBQ = kBD + 2 * kDR;
   auto b_q_full = [&](int s) { return bar0 + 8u * (kBQ + s); };
   auto b_q_empty = [&](int s) { return bar0 + 8u * (kBQ + C::kQS + s); };
   const uint32_t b_mma_done = bar0 + 8u * (kBQ + 2 * C::kQS);
   PPMisc* misc = reinterpret_cast<PPMisc*>(smem + C::kOffMisc);
   volatile int* abort_flag = &misc->abort;
   volatile int* vdec = &misc->dec[0][0];
+  // wait for commit number i of row block t (bounded)
+  auto wait_cm = [&](int t, int i) {
+    return mbar_wait(b_cm(t, i), (i / kCR) & 1, abort_flag, wait_limit_ns);
+  };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -173,25 +211,18 @@ __global__ void __launch_bounds__(kPPThreads, 1)
   const long long n_items = static_cast<long long>(BH) * n_pairs;
 
   if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kKS; ++s) mbar_init(b_k_full(s), 1);
+    for (int s = 0; s < C::kVS; ++s) mbar_init(b_v_full(s), 1);
+    for (int t = 0; t < 2; ++t) {
+      for (int i = 0; i < kCR; ++i) mbar_init(b_cm(t, i), 1);
+      for (int b = 0; b < SB; ++b) mbar_init(b_p_full(t, b), 4);
+      for (int i = 0; i < kDR; ++i) mbar_init(b_dec(t, i), 1);
+    }
     for (int s = 0; s < C::kQS; ++s) {
       mbar_init(b_q_full(s), 1);
       mbar_init(b_q_empty(s), 1);
     }
     mbar_init(b_mma_done, 1);
-    for (int s = 0; s < C::kKS; ++s) {
-      mbar_init(b_k_full(s), 1);
-      mbar_init(b_k_empty(s), 1);
-    }
-    for (int s = 0; s < C::kVS; ++s) {
-      mbar_init(b_v_full(s), 1);
-      mbar_init(b_v_empty(s), 1);
-    }
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(b_s_full(t), 1);
-      mbar_init(b_p_full(t), 4);
-      mbar_init(b_o_full(t), 1);
-      for (int i = 0; i < kDR; ++i) mbar_init(b_dec(t, i), 1);
-    }
     misc->abort = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -205,13 +236,16 @@ __global__ void __launch_bounds__(kPPThreads, 1)
   tc_fence_after();
   const uint32_t tmem = misc->tmem_base;
   auto tO = [&](int t) { return tmem + t * D; };
-  auto tS = [&](int t) { return tmem + 2 * D + t * BC; };
+  auto tS = [&](int t, int b) { return tmem + 2 * D + (t * SB + b) * BC; };
 
   if (warp < 4) {
     reg_dec<C::kProducerRegs>();
     if (warp == 0 && lane == 0) {
       // ---------------------------------------------------- Q and K producer
       int kload = 0, items = 0, kdone = 0;
+      int base0 = 0, base1 = 0;  // commit counts of earlier items, per row block
+      Pending3 pend;
+      pend.init();
       bool alive = true;
       for (long long idx = blockIdx.x; alive && idx < n_items; idx += gridDim.x, ++items) {
         const Item it = make_item<BC, CAUSAL>(idx, BH, n_pairs, n_rb, N);
@@ -230,18 +264,25 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                         p * 64, (it.rb0 + t) * kRows, it.bh);
         for (int j = 0; j < it.Tmax; ++j) {
           const int s = kload % C::kKS;
-          if (kload >= C::kKS &&
-              !mbar_wait(b_k_empty(s), ((kload / C::kKS) - 1) & 1, abort_flag, wait_limit_ns)) {
-            pp_give_up(misc, status, 2);
-            alive = false;
-            break;
+          if (pend.n == C::kKS) {  // the slot's previous tile: its S MMAs must have run
+            if (!wait_cm(pend.r[0], pend.c[0])) {
+              pp_give_up(misc, status, 2);
+              alive = false;
+              break;
+            }
+            pend.pop();
           }
           mbar_arrive_expect_tx(b_k_full(s), C::kKVBytes);
           for (int p = 0; p < C::kPanels; ++p)
             tma_load_3d(sK + s * C::kKVBytes + p * C::kKVPanel, &tmK, b_k_full(s), p * 64, j * BC,
                         bkv);
+          // K tile j is read by S of row block 1 last (if it exists, T1 >= T0)
+          if (j < it.T1) pend.push(1, base1 + j, 0);
+          else pend.push(0, base0 + j, 0);
           ++kload;
         }
+        base0 += commits_of<SB>(it.T0);
+        base1 += commits_of<SB>(it.T1);
         kdone = items + 1;
       }
       // never leave with a copy in flight
@@ -253,25 +294,41 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       // ---------------------------------------------------- V producer
       int vload = 0;
       int dl[2] = {0, 0};
+      int base0 = 0, base1 = 0;
+      int gbase = 0;  // running tile number of this item's key tile 0
+      Pending3 pend;
+      pend.init();
       bool alive = true;
-      auto issue_v = [&](int j, int bkv) -> bool {
-        const int s = vload % C::kVS;
-        if (vload >= C::kVS &&
-            !mbar_wait(b_v_empty(s), ((vload / C::kVS) - 1) & 1, abort_flag, wait_limit_ns))
-          return false;
-        mbar_arrive_expect_tx(b_v_full(s), C::kKVBytes);
-        for (int p = 0; p < C::kPanels; ++p)
-          tma_load_3d(sV + s * C::kKVBytes + p * C::kKVPanel, &tmV, b_v_full(s), p * 64, j * BC, bkv);
-        ++vload;
-        return true;
-      };
       for (long long idx = blockIdx.x; alive && idx < n_items; idx += gridDim.x) {
         const Item it = make_item<BC, CAUSAL>(idx, BH, n_pairs, n_rb, N);
         const int bkv = (it.bh / Hq) * Hkv + (it.bh % Hq) / g;
         const int T[2] = {it.T0, it.T1};
+        auto issue_v = [&](int j) -> bool {
+          if (pend.n == C::kVS) {
+            // The slot's previous tile: its P*V MMAs must have run.  Once a
+            // decision on tile j has been read, S_j has completed, and with
+            // it every MMA issued before it: all P*V of tiles j - SB - 1 and
+            // earlier (items are SB apart in g).  Those commits are not
+            // waited for, since their ring slot may have been reused after a
+            // run of skipped tiles.
+            const bool known_done = !tau_is_inf && pend.g[0] + SB < gbase + j;
+            if (!known_done && !wait_cm(pend.r[0], pend.c[0])) return false;
+            pend.pop();
+          }
+          const int s = vload % C::kVS;
+          mbar_arrive_expect_tx(b_v_full(s), C::kKVBytes);
+          for (int p = 0; p < C::kPanels; ++p)
+            tma_load_3d(sV + s * C::kKVBytes + p * C::kKVPanel, &tmV, b_v_full(s), p * 64, j * BC,
+                        bkv);
+          // P*V of tile j, row block 1 (if it visits j) is issued after row block 0's
+          if (j < it.T1) pend.push(1, base1 + min(SB, it.T1) + j, gbase + j);
+          else pend.push(0, base0 + min(SB, it.T0) + j, gbase + j);
+          ++vload;
+          return true;
+        };
         for (int j = 0; alive && j < it.Tmax; ++j) {
           if (tau_is_inf) {
-            if (!issue_v(j, bkv)) {
+            if (!issue_v(j)) {
               pp_give_up(misc, status, 4);
               alive = false;
             }
@@ -282,25 +339,27 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           bool issued = false;
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
-            if (!alive) break;
-            if (j >= T[t]) continue;
+            if (!alive || j >= T[t]) continue;
             const int di = dl[t] % kDR;
             if (!mbar_wait(b_dec(t, di), (dl[t] / kDR) & 1, abort_flag, wait_limit_ns)) {
               pp_give_up(misc, status, 3);
               alive = false;
-              break;
+              continue;
             }
             ++dl[t];
             if (vdec[t * kDR + di] && !issued) {
-              if (!issue_v(j, bkv)) {
+              if (!issue_v(j)) {
                 pp_give_up(misc, status, 4);
                 alive = false;
-                break;
+                continue;
               }
               issued = true;
             }
           }
         }
+        base0 += commits_of<SB>(it.T0);
+        base1 += commits_of<SB>(it.T1);
+        gbase += it.Tmax + SB;
       }
       for (int t = max(0, vload - C::kVS); t < vload; ++t)
         mbar_drain(b_v_full(t % C::kVS), (t / C::kVS) & 1, wait_limit_ns);
@@ -309,24 +368,28 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       constexpr uint32_t idS = idesc_bf16_f32(kRows, BC, false, false);
       constexpr uint32_t idPV = idesc_bf16_f32(kRows, D, false, true);
       int kuse = 0, vuse = 0, items = 0;
-      int pc[2] = {0, 0}, dc[2] = {0, 0};
+      int pc[2] = {0, 0}, dc[2] = {0, 0}, sq[2] = {0, 0}, cmc[2] = {0, 0};
       bool alive = true;
       // Descriptors differ only in their start-address field (bits 0-13, in
-      // 16-byte units), so each MMA adds a compile-time offset to a base.
+      // 16-byte units): each MMA adds a compile-time offset to a 32-bit base.
       constexpr uint32_t kHi = sw128_desc_hi(1024);
       const uint32_t dK0 = sw128_desc_lo(sK, 16);
       const uint32_t dV0 = sw128_desc_lo(sV, C::kKVPanel);
       uint32_t dQ = sw128_desc_lo(sQ, 16);  // this item's Q slot
-      auto issue_S = [&](int t, int kslot) {
+      auto issue_S = [&](int t, int kslot, int buf) {
         const uint32_t a0 = dQ + t * (C::kQTile >> 4);
         const uint32_t b0 = dK0 + kslot * (C::kKVBytes >> 4);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t oq = ((kk >> 2) * C::kQPanel + (kk & 3) * 32) >> 4;
           const uint32_t ok_ = ((kk >> 2) * C::kKVPanel + (kk & 3) * 32) >> 4;
-          mma_ss(tS(t), desc_join(a0 + oq, kHi), desc_join(b0 + ok_, kHi), idS, kk > 0 ? 1u : 0u);
+          mma_ss(tS(t, buf), desc_join(a0 + oq, kHi), desc_join(b0 + ok_, kHi), idS,
+                 kk > 0 ? 1u : 0u);
         }
-        mma_commit(b_s_full(t));
+      };
+      auto commit = [&](int t) {
+        mma_commit(b_cm(t, cmc[t]));
+        ++cmc[t];
       };
       for (long long idx = blockIdx.x; alive && idx < n_items; idx += gridDim.x, ++items) {
         const Item it = make_item<BC, CAUSAL>(idx, BH, n_pairs, n_rb, N);
@@ -337,29 +400,37 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           pp_give_up(misc, status, 5);
           break;
         }
-        // prologue: S_t_0
-        if (!mbar_wait(b_k_full(kuse % C::kKS), (kuse / C::kKS) & 1, abort_flag, wait_limit_ns)) {
-          pp_give_up(misc, status, 6);
-          break;
-        }
-        tc_fence_after();
+        // prologue: S of the first SB key tiles, one commit per row block and tile
+        for (int jj = 0; alive && jj < SB && jj < it.Tmax; ++jj) {
+          if (!mbar_wait(b_k_full(kuse % C::kKS), (kuse / C::kKS) & 1, abort_flag, wait_limit_ns)) {
+            pp_give_up(misc, status, 6);
+            alive = false;
+            break;
+          }
+          tc_fence_after();
 #pragma unroll
-        for (int t = 0; t < 2; ++t)
-          if (T[t] > 0) issue_S(t, kuse % C::kKS);
-        mma_commit(b_k_empty(kuse % C::kKS));
-        ++kuse;
+          for (int t = 0; t < 2; ++t)
+            if (jj < T[t]) {
+              issue_S(t, kuse % C::kKS, sq[t] % SB);
+              ++sq[t];
+              commit(t);
+            }
+          ++kuse;
+        }
+        if (!alive) break;
         // the Q slot is free once the item's last S MMA has run
-        if (it.Tmax == 1) mma_commit(b_q_empty(qs));
+        if (it.Tmax <= SB) mma_commit(b_q_empty(qs));
         bool started[2] = {false, false};
         for (int j = 0; alive && j < it.Tmax; ++j) {
           bool v_used = false, k_next = false;
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
-            if (j >= T[t]) continue;
-            if (!mbar_wait(b_p_full(t), pc[t] & 1, abort_flag, wait_limit_ns)) {
+            if (!alive || j >= T[t]) continue;
+            const int pb = pc[t] % SB;
+            if (!mbar_wait(b_p_full(t, pb), (pc[t] / SB) & 1, abort_flag, wait_limit_ns)) {
               pp_give_up(misc, status, 7);
               alive = false;
-              break;
+              continue;
             }
             ++pc[t];
             tc_fence_after();
@@ -371,7 +442,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                                wait_limit_ns)) {
                   pp_give_up(misc, status, 8);
                   alive = false;
-                  break;
+                  continue;
                 }
                 tc_fence_after();
                 v_used = true;
@@ -379,34 +450,30 @@ __global__ void __launch_bounds__(kPPThreads, 1)
               const uint32_t vb = dV0 + (vuse % C::kVS) * (C::kKVBytes >> 4);
 #pragma unroll
               for (int kk = 0; kk < BC / 16; ++kk)
-                mma_ts(tO(t), tS(t) + kk * 8, desc_join(vb + ((kk * 16 * 128) >> 4), kHi), idPV,
+                mma_ts(tO(t), tS(t, pb) + kk * 8, desc_join(vb + ((kk * 16 * 128) >> 4), kHi), idPV,
                        (started[t] || kk > 0) ? 1u : 0u);
               started[t] = true;
             }
-            if (j == T[t] - 1) mma_commit(b_o_full(t));
-            if (j + 1 < T[t]) {
+            // S for key tile j + SB reuses the buffer P_t_j just left
+            if (j + SB < T[t]) {
               if (!k_next) {
                 if (!mbar_wait(b_k_full(kuse % C::kKS), (kuse / C::kKS) & 1, abort_flag,
                                wait_limit_ns)) {
                   pp_give_up(misc, status, 9);
                   alive = false;
-                  break;
+                  continue;
                 }
                 tc_fence_after();
                 k_next = true;
               }
-              issue_S(t, kuse % C::kKS);
+              issue_S(t, kuse % C::kKS, sq[t] % SB);
+              ++sq[t];
             }
+            commit(t);  // #(base_t + min(SB, T_t) + j): P*V_t_j and S_t_{j+SB}
           }
-          if (k_next) {
-            mma_commit(b_k_empty(kuse % C::kKS));
-            ++kuse;
-          }
-          if (j + 2 == it.Tmax) mma_commit(b_q_empty(qs));  // S MMAs of tile Tmax-1 issued
-          if (v_used) {
-            mma_commit(b_v_empty(vuse % C::kVS));
-            ++vuse;
-          }
+          if (k_next) ++kuse;
+          if (v_used) ++vuse;
+          if (j + SB + 1 == it.Tmax) mma_commit(b_q_empty(qs));  // last S MMAs issued
         }
       }
       // all issued MMAs must finish before TMEM is released
@@ -416,17 +483,19 @@ __global__ void __launch_bounds__(kPPThreads, 1)
   } else {
     reg_inc<C::kSoftmaxRegs>();
     // -------------------------------------------------------- softmax warpgroups
-    const int t = (warp - 4) >> 2;    // row block of the pair
-    const int sw = warp & 3;          // TMEM sub-partition of this warp
+    const int t = (warp - 4) >> 2;  // row block of the pair
+    const int sw = warp & 3;        // TMEM sub-partition of this warp
     const int row = sw * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(sw * 32) << 16;
     const float NEG_INF = -__int_as_float(0x7f800000);
-    int sc = 0, dcount = 0, oc = 0;
+    int sc = 0, dcount = 0;
+    int base = 0;  // this row block's commits in earlier items
     bool ok = true, failed = false;
     for (long long idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
       const Item it = make_item<BC, CAUSAL>(idx, BH, n_pairs, n_rb, N);
       const int T = t == 0 ? it.T0 : it.T1;
       if (T == 0) continue;  // this row block does not exist
+      const int pro = min(SB, T);
       const int rb = it.rb0 + t;
       const int q_idx = rb * kRows + row;
       const bool row_valid = q_idx < N;
@@ -434,16 +503,16 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           skip_mask ? ((static_cast<size_t>(it.bh) * n_rb + rb) * n_tiles) : 0;
       float m_exact = NEG_INF, m_ref = NEG_INF, l_sum = 0.f;
       for (int j = 0; j < T; ++j) {
-        bool waited = !failed && __all_sync(0xffffffffu, mbar_wait(b_s_full(t), sc & 1, abort_flag,
-                                                                     wait_limit_ns));
+        const int sb = sc % SB;  // S/P buffer of key tile j
         ++sc;
+        bool waited = !failed && __all_sync(0xffffffffu, wait_cm(t, base + j));
         // raw scores stay in registers as fp32 bit patterns; the log2 scale is
         // folded into the max (positive scale) and into the exp FFMA below
         uint32_t u[BC];
         float mt = NEG_INF;
         if (waited) {
           tc_fence_after();
-          tmem_ld_row<BC>(tS(t) + lane_off, u);
+          tmem_ld_row<BC>(tS(t, sb) + lane_off, u);
           tmem_wait_ld();
           // last visible column of this row in tile j (-1: none); one integer
           // limit keeps the masking to a compare-select per column
@@ -501,10 +570,10 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         }
         if (skip) {
           __syncwarp();
-          if (lane == 0) mbar_arrive(b_p_full(t));
+          if (lane == 0) mbar_arrive(b_p_full(t, sb));
           continue;
         }
-        // ---- kept tile: lazy reference max, O rescale (O_t is idle here), P
+        // ---- kept tile: lazy reference max, P, then O rescale
         const float m_cand = fmaxf(m_ref, mt);
         const bool moved = row_valid && (m_cand > m_ref + kRescale);
         float alpha = 1.f;
@@ -530,37 +599,48 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             rs2 = __fadd2_rn(rs2, make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)));
             pk[c] = w;
           }
-          tmem_st16(tS(t) + lane_off + c0 / 2, pk);
+          tmem_st16(tS(t, sb) + lane_off + c0 / 2, pk);
         }
-        const float rs = rs2.x + rs2.y;
-        l_sum = l_sum * alpha + rs;
-        // O_t is idle (S_t_j done => PV_t_{j-1} done); rescale after the P
-        // store so the scores are no longer live
+        l_sum = l_sum * alpha + (rs2.x + rs2.y);
+        // O rescale (after the P store, so the scores are no longer live).
+        // P*V of tile j-1 must have finished: commit #(base + pro + j - 1).
+        // With one S buffer that is the commit S_j already waited for.
         if (j > 0 && __any_sync(0xffffffffu, moved)) {
-          tc_fence_after();
-          const float a = moved ? alpha : 1.f;
+          if (SB > 1 && !__all_sync(0xffffffffu, wait_cm(t, base + pro + j - 1))) {
+            pp_give_up(misc, status, 12);
+            failed = true;  // acted on at the next vote, or just below
+          }
+          if (!failed) {
+            tc_fence_after();
+            const float a = moved ? alpha : 1.f;
 #pragma unroll
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t r[32];
-            tmem_ld32(tO(t) + lane_off + c0, r);
-            tmem_wait_ld();
+            for (int c0 = 0; c0 < D; c0 += 32) {
+              uint32_t r[32];
+              tmem_ld32(tO(t) + lane_off + c0, r);
+              tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * a);
-            tmem_st32(tO(t) + lane_off + c0, r);
+              for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(__uint_as_float(r[c]) * a);
+              tmem_st32(tO(t) + lane_off + c0, r);
+            }
           }
         }
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(b_p_full(t));
+        if (lane == 0) mbar_arrive(b_p_full(t, sb));
+        if (failed && tau_is_inf) {  // no votes without a finite tau: stop here
+          ok = false;
+          break;
+        }
       }
+      if (failed) ok = false;
       if (!ok) break;
       // ---- epilogue: O / l -> bf16 -> global; unvisited tiles marked 2
       if (skip_mask)
         for (int j = T + row; j < n_tiles; j += 128) skip_mask[mask_base + j] = 2;
-      const bool done =
-          __all_sync(0xffffffffu, mbar_wait(b_o_full(t), oc & 1, abort_flag, wait_limit_ns));
-      ++oc;
+      // P*V of the last tile finished: commit #(base + pro + T - 1)
+      const bool done = __all_sync(0xffffffffu, wait_cm(t, base + pro + T - 1));
+      base += pro + T;
       if (!done) {
         pp_give_up(misc, status, 11);
         ok = false;
