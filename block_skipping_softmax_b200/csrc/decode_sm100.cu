@@ -9,22 +9,36 @@
 // KV head, because they share the V tile that a skip avoids reading.
 //
 // Work split: CTA (split, kv head, batch) streams its split's 64-key tiles.
-// Decode is bound by HBM reads of K and V, so the kernel is built around the
-// memory system rather than the tensor cores (a g-row GEMV does not fill an
-// MMA): every K tile is one contiguous 16 KB (d=128) bulk copy into a shared-
-// memory ring, issued three tiles ahead; a V tile is requested only once the
-// tile is known to be kept, and consumed two iterations later so its latency
-// stays hidden.  Shared memory is read with 16-byte vector loads, each warp
-// instruction covering whole key rows; dot products use packed fp32 FMAs and
-// a transposing butterfly reduction across the lanes of one key.
+// Decode is bound by HBM reads of K and V; a g-row GEMV does not fill an MMA,
+// so the arithmetic runs on the FMA pipes and the design goal is the fewest
+// issued instructions per byte, so that the memory system stays the limit:
 //
-// One CTA barrier per tile: the scores of tile i and each warp's per-row
-// maxima are formed before it; after it every thread takes the same skip
-// decision from the eight warp maxima (no serial phase), the lanes that hold
-// scores turn them into probabilities for a later P*V, and thread 0 refills
-// the copy rings.  Output per split: normalised partial o (fp32) and its
-// log2-sum-exp; a second kernel merges the splits exactly.
+//  * Tiles arrive by TMA as 64-column panels with the 128-byte swizzle (16 KB
+//    per d=128 tile), K three tiles ahead of the compute; a V tile is
+//    requested only once its tile is known to be kept and is consumed two
+//    iterations later.  The swizzle lets a group of eight lanes read eight
+//    different keys (or eight chunks of one key) without bank conflicts, so
+//    each lane can hold several 16-byte chunks of a key row and the cross-lane
+//    reduction of a score shrinks to a few butterfly steps.
+//  * Scores: kP lanes share a key, each with kCPL chunks of q and k in fp32,
+//    packed FMAs; the butterfly transposes so that a lane ends up with the
+//    score of one (key, query row).  The 1/sqrt(d) and log2(e) factors are
+//    folded into q.
+//  * One CTA barrier per tile.  After it every warp takes the same skip
+//    decision lane-parallel (lane = one (warp, row) maximum, a 3-step max
+//    butterfly, one vote), so no warp waits on a serial decision phase.
+//  * A lazy reference max per row: probabilities are taken relative to a
+//    value that is moved up only when the running max exceeds it by more
+//    than 2^8, so the partial sums are rescaled rarely.  The skip test itself
+//    always uses the exact running max.
+//  * P*V: a thread owns one 16-byte chunk of d for all g rows and a fixed
+//    subset of the tile's keys; the sums over key subsets are combined once
+//    at the end of the split.
+//
+// Output per split: normalised partial o (fp32) and its log2-sum-exp; a second
+// kernel merges the splits exactly.
 #include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -43,42 +57,101 @@ constexpr int kKStages = 3;  // K tiles in flight ahead of the compute
 constexpr int kLag = 2;      // a kept tile's P*V runs kLag iterations after its test
 constexpr int kVStages = kLag + 1;
 constexpr int kPRing = kLag + 1;
+constexpr float kRefSlack = 8.f;  // log2 units: probabilities stay below 2^8
 
 template <int D, int G>
 struct DecCfg {
-  static constexpr int kTileBytes = kDecodeTile * D * 2;
-  static constexpr int kCPK = D / 8;                  // 16-byte chunks per key row
-  static constexpr int kKPI = 32 / kCPK;              // keys per warp instruction
+  static constexpr int kPanels = D / 64;                 // 64-column panels per key row
+  static constexpr int kPanelBytes = kDecodeTile * 128;  // 64 keys x 128 B
+  static constexpr int kTileBytes = kPanels * kPanelBytes;
+  static constexpr int kChunks = D / 8;  // 16-byte chunks per key row
+  // score phase: kP lanes share a key, each holding kCPL chunks of q (at most
+  // 64 fp32 values of q per lane)
+  static constexpr int kCPL = (kChunks / 4 < 8 / G) ? kChunks / 4 : 8 / G;
+  static constexpr int kP = kChunks / kCPL;
+  static constexpr int kKPI = 32 / kP;                 // keys per warp instruction
   static constexpr int kKeysPerWarp = kDecodeTile / kWarps;
-  static constexpr int kIters = kKeysPerWarp / kKPI;
-  static constexpr int kLanesPerRow = kCPK / G;       // lanes holding copies of one score
+  static constexpr int kSIters = kKeysPerWarp / kKPI;  // score iterations per tile
+  static constexpr bool kKeyMajor = kP >= 8;           // lane = key * kP + qd, else qd * kKPI + key
+  static constexpr int kDup = kP / G;                  // lanes holding the same (key, row) score
+  // P*V phase: kChunks lanes per key, kGroups disjoint key subsets
+  static constexpr int kGroups = kDecThreads / kChunks;
+  static constexpr int kVKeys = kDecodeTile / kGroups;
+  // shared memory (offsets from a 1024-byte aligned base)
   static constexpr int kOffK = 0;
   static constexpr int kOffV = kOffK + kKStages * kTileBytes;
-  static constexpr int kOffP = kOffV + kVStages * kTileBytes;             // float [PR][64][G]
-  static constexpr int kOffW = kOffP + kPRing * kDecodeTile * G * 4;      // float [2][warps][G]
-  static constexpr int kOffMisc = kOffW + 2 * kWarps * G * 4;
-  static constexpr int kOffBar = kOffMisc + 64;                           // k_full, v_full
-  static constexpr int kSmemBytes = kOffBar + 8 * (kKStages + kVStages) + 128;
-  // the final cross-warp reduction reuses the K ring
-  static_assert(kWarps * G * (D + 1) * 4 <= kKStages * kTileBytes, "reduction scratch");
-  static_assert(G <= kCPK, "rows per group");
+  static constexpr int kOffP = kOffV + kVStages * kTileBytes;          // float [ring][64][G]
+  static constexpr int kOffR = kOffP + kPRing * kDecodeTile * G * 4;   // float [ring][8] ref max
+  static constexpr int kOffF = kOffR + kPRing * 8 * 4;                 // int [ring] rescale flag
+  static constexpr int kOffW = kOffF + 16;                             // float [2][warps][G]
+  static constexpr int kOffL = kOffW + 2 * kWarps * G * 4;             // float [warps][G]
+  static constexpr int kOffMisc = kOffL + kWarps * G * 4;
+  static constexpr int kOffBar = kOffMisc + 16;
+  static constexpr int kSmemUsed = kOffBar + 8 * (kKStages + kVStages);
+  static constexpr int kSmemBytes = kSmemUsed + 1024;  // room to align the base
+  static_assert(G <= kP, "a lane ends the butterfly with one row");
+  static_assert(kSIters >= 1 && kKPI * kSIters == kKeysPerWarp, "score lane layout");
+  static_assert(kKeyMajor || kKPI == 8, "qd-major lanes need eight keys per instruction");
+  static_assert(kChunks >= 8 && kGroups * kVKeys == kDecodeTile, "P*V lane layout");
+  static_assert(kWarps * G * D * 4 <= kKStages * kTileBytes, "reduction scratch");
+  static_assert(G <= 8 && kOffP % 16 == 0, "ring layout");
 };
+
+constexpr int ilog2(int x) { return x <= 1 ? 0 : 1 + ilog2(x / 2); }
+
+// byte offset of 16-byte chunk `lc` of key row `k` in a tile of swizzled panels
+template <int D>
+__device__ __forceinline__ uint32_t chunk_off(int k, int lc) {
+  return static_cast<uint32_t>((lc >> 3) * (kDecodeTile * 128) + k * 128 +
+                               (((lc & 7) ^ (k & 7)) << 4));
+}
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 u, float2 (&f)[4]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int e = 0; e < 4; ++e)
+    f[e] = make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xffff0000u));
+}
+
+template <int G>
+__device__ __forceinline__ void load_row_floats(const float* p, float (&v)[G]) {
+  if constexpr (G % 4 == 0) {
+#pragma unroll
+    for (int i = 0; i < G; i += 4) {
+      const float4 x = *reinterpret_cast<const float4*>(p + i);
+      v[i] = x.x; v[i + 1] = x.y; v[i + 2] = x.z; v[i + 3] = x.w;
+    }
+  } else if constexpr (G == 2) {
+    const float2 x = *reinterpret_cast<const float2*>(p);
+    v[0] = x.x; v[1] = x.y;
+  } else {
+    v[0] = p[0];
+  }
+}
 
 }  // namespace
 
 template <int D, int G>
 __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
-    decode_partial_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ K,
-                          const __nv_bfloat16* __restrict__ V, float* __restrict__ o_part,
+    decode_partial_kernel(const __grid_constant__ CUtensorMap tmK,
+                          const __grid_constant__ CUtensorMap tmV,
+                          const __nv_bfloat16* __restrict__ q, float* __restrict__ o_part,
                           float* __restrict__ lse_part, uint8_t* __restrict__ skip_mask,
                           int* __restrict__ status, int Hq, int Hkv, int L, int split_len,
                           int n_splits, float scale_log2, float tau_log2, int tau_is_inf,
                           unsigned long long wait_limit_ns) {
   using C = DecCfg<D, G>;
-  extern __shared__ __align__(128) uint8_t smem[];
-  const uint32_t sbase = smem_u32(smem);
+  constexpr unsigned FULL = 0xffffffffu;
+  constexpr int kLog2P = ilog2(C::kP);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;  // the swizzle pattern repeats every 1024 B
+  uint8_t* smem = smem_raw + (sbase - raw);
   float* p_ring = reinterpret_cast<float*>(smem + C::kOffP);
+  float* ref_ring = reinterpret_cast<float*>(smem + C::kOffR);
+  int* flag_ring = reinterpret_cast<int*>(smem + C::kOffF);
   float* wmax = reinterpret_cast<float*>(smem + C::kOffW);
+  float* wl = reinterpret_cast<float*>(smem + C::kOffL);
   // Give-ups are made CTA-uniform with __syncthreads_or, so no role ever
   // needs to be told to stop early: this flag stays 0.
   volatile int* never = reinterpret_cast<volatile int*>(smem + C::kOffMisc);
@@ -92,18 +165,19 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
   const int split = blockIdx.x;
   const int kv = blockIdx.y;
   const int b = blockIdx.z;
+  const int bh = b * Hkv + kv;
   const int n_tiles_all = (L + kDecodeTile - 1) / kDecodeTile;
   const int t_begin = split * (split_len / kDecodeTile);
   const int t_end = min(n_tiles_all, t_begin + split_len / kDecodeTile);
   const int nt = t_end - t_begin;
-  const size_t kv_off = (static_cast<size_t>(b) * Hkv + kv) * static_cast<size_t>(L) * D;
-  const __nv_bfloat16* Kg = K + kv_off;
-  const __nv_bfloat16* Vg = V + kv_off;
   const float NEG_INF = -__int_as_float(0x7f800000);
 
-  auto tile_bytes = [&](int t) {  // the last tile of the sequence may be ragged
-    const int keys = min(kDecodeTile, L - t * kDecodeTile);
-    return static_cast<uint32_t>(keys * D * 2);
+  // one tile = kPanels TMA boxes of 64 columns x 64 keys; rows past L read as zeros
+  auto issue = [&](uint32_t dst, const CUtensorMap* map, uint32_t bar, int t) {
+    mbar_arrive_expect_tx(bar, C::kTileBytes);
+#pragma unroll
+    for (int p = 0; p < C::kPanels; ++p)
+      tma_load_3d(dst + p * C::kPanelBytes, map, bar, p * 64, t * kDecodeTile, bh);
   };
 
   if (tid == 0) {
@@ -117,44 +191,47 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
   int k_issued = 0, v_issued = 0;
   if (tid == 0) {
     for (int i = 0; i < kKStages && i < nt; ++i) {
-      const int t = t_begin + i;
-      mbar_arrive_expect_tx(b_k_full(i), tile_bytes(t));
-      bulk_load(sbase + C::kOffK + i * C::kTileBytes, Kg + static_cast<size_t>(t) * kDecodeTile * D,
-                tile_bytes(t), b_k_full(i));
+      issue(sbase + C::kOffK + i * C::kTileBytes, &tmK, b_k_full(i), t_begin + i);
       ++k_issued;
     }
   }
 
-  // this lane's slice: 16-byte chunk `c` of key `sub` within each warp instruction
-  const int c = lane % C::kCPK;
-  const int sub = lane / C::kCPK;
-  const int my_row = c / C::kLanesPerRow;  // the score row this lane ends up holding
-  const bool writer = (c % C::kLanesPerRow) == 0;
-  float2 qf[G][4];
+  // score-phase roles: lane holds chunks lc = j*kP + qd of key kl; after the
+  // butterfly it holds the score of (key, row_q)
+  const int qd = C::kKeyMajor ? (lane % C::kP) : (lane / C::kKPI);
+  const int kl = C::kKeyMajor ? (lane / C::kP) : (lane % C::kKPI);
+  const int row_q = qd / C::kDup;
+  const bool leader = (qd % C::kDup) == 0;
+  // P*V roles: chunk ch of d, keys kg + kGroups*e
+  const int ch = lane % C::kChunks;
+  const int kg = warp * (32 / C::kChunks) + lane / C::kChunks;
+  // decision roles: lane < n_dec holds the maximum of (warp lane/G, row lane%G)
+  constexpr int n_dec = (8 * G < 32) ? 8 * G : 32;
+
+  float2 qf[G][C::kCPL][4];
 #pragma unroll
   for (int r = 0; r < G; ++r) {
-    const uint4 u = *reinterpret_cast<const uint4*>(
-        q + (static_cast<size_t>(b) * Hq + kv * G + r) * D + c * 8);
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-    for (int e = 0; e < 4; ++e)
-      qf[r][e] = make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xffff0000u));
+    for (int j = 0; j < C::kCPL; ++j) {
+      const uint4 u = *reinterpret_cast<const uint4*>(
+          q + (static_cast<size_t>(b) * Hq + kv * G + r) * D + (j * C::kP + qd) * 8);
+      bf16x8_to_f32(u, qf[r][j]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        qf[r][j][e] = __fmul2_rn(qf[r][j][e], make_float2(scale_log2, scale_log2));
+    }
   }
-  float2 acc[G][4];
-  float lsum[G];
-  // every thread keeps identical copies of the decision state
-  float m_exact[G];           // exact running max after the latest tested tile (log2 units)
-  float m_hist[kLag + 1][G];  // m_hist[k][r] = running max after tile i - k
-  float m_acc[G];             // reference max of the partial sums acc / lsum
+
+  float m_exact = NEG_INF;  // decision lanes: exact running max of row lane % G (log2 units)
+  float m_ref = NEG_INF;    // decision lanes: reference max of that row
+  float lsum = 0.f;         // leader score lanes: sum of p for row row_q over this lane's keys
+  float2 acc[G][4];         // P*V threads: rows x 8 columns of chunk ch
+  float m_acc[G];           // P*V threads: reference max the sums in acc are relative to
 #pragma unroll
   for (int r = 0; r < G; ++r) {
-    lsum[r] = 0.f;
-    m_exact[r] = NEG_INF;
     m_acc[r] = NEG_INF;
 #pragma unroll
     for (int e = 0; e < 4; ++e) acc[r][e] = make_float2(0.f, 0.f);
-#pragma unroll
-    for (int k = 0; k <= kLag; ++k) m_hist[k][r] = NEG_INF;
   }
   uint32_t kept_bits = 0;  // bit k: tile i - k was kept
   int pv_count = 0;        // V tiles consumed
@@ -162,123 +239,124 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
 
   for (int i = 0; i < nt + kLag; ++i) {
     // ---------------- A: scores of tile i and the per-warp row maxima
-    float sv[C::kIters];
+    float sv[C::kSIters];
     if (i < nt) {
       const int ks = i % kKStages;
       const bool got = mbar_wait(b_k_full(ks), (i / kKStages) & 1, never, wait_limit_ns);
-      ok = ok && got;
+      ok = ok && got;  // on a give-up the scores are garbage and dropped at the barrier
       const uint8_t* kt = smem + C::kOffK + ks * C::kTileBytes;
       const int key_lim = L - (t_begin + i) * kDecodeTile;  // keys >= key_lim are past L
       float wm = NEG_INF;
 #pragma unroll
-      for (int it = 0; it < C::kIters; ++it) {
-        const int key = warp * C::kKeysPerWarp + it * C::kKPI + sub;
-        float v[G];
-        if (got) {
-          const uint4 u = *reinterpret_cast<const uint4*>(kt + key * D * 2 + c * 16);
-          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+      for (int it = 0; it < C::kSIters; ++it) {
+        const int key = warp * C::kKeysPerWarp + it * C::kKPI + kl;
+        float2 s2[G];
+#pragma unroll
+        for (int r = 0; r < G; ++r) s2[r] = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int j = 0; j < C::kCPL; ++j) {
+          const uint4 u = *reinterpret_cast<const uint4*>(kt + chunk_off<D>(key, j * C::kP + qd));
           float2 kf[4];
+          bf16x8_to_f32(u, kf);
 #pragma unroll
-          for (int e = 0; e < 4; ++e)
-            kf[e] = make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xffff0000u));
+          for (int r = 0; r < G; ++r)
 #pragma unroll
-          for (int r = 0; r < G; ++r) {
-            float2 s2 = __fmul2_rn(qf[r][0], kf[0]);
-#pragma unroll
-            for (int e = 1; e < 4; ++e) s2 = __ffma2_rn(qf[r][e], kf[e], s2);
-            v[r] = s2.x + s2.y;
-          }
-        } else {
-#pragma unroll
-          for (int r = 0; r < G; ++r) v[r] = 0.f;
+            for (int e = 0; e < 4; ++e) s2[r] = __ffma2_rn(qf[r][j][e], kf[e], s2[r]);
         }
-        // transposing butterfly over the kCPK lanes of this key: each halving
-        // step keeps half of the rows, so after log2(G) steps a lane owns one
-        // row (my_row); the remaining steps are plain sums
+        float v[G];
 #pragma unroll
-        for (int step = 0; (C::kCPK >> (step + 1)) >= 1; ++step) {
-          const int o = C::kCPK >> (step + 1);
-          const int n = G >> step;
+        for (int r = 0; r < G; ++r) v[r] = s2[r].x + s2[r].y;
+        // butterfly over the kP lanes of this key, highest qd bit first: the
+        // first log2(G) steps each keep half of the rows (the lanes with the
+        // bit set keep the upper half), the rest are plain sums
+#pragma unroll
+        for (int s = 0; s < kLog2P; ++s) {
+          const int qbit = kLog2P - 1 - s;
+          const int o = C::kKeyMajor ? (1 << qbit) : (C::kKPI << qbit);
+          const int n = G >> s;
           if (n > 1) {
             const int hh = n / 2;
-            const bool upper = (lane & o) != 0;
+            const bool upper = ((qd >> qbit) & 1) != 0;
 #pragma unroll
             for (int r = 0; r < hh; ++r) {
               const float send = upper ? v[r] : v[r + hh];
               const float keep = upper ? v[r + hh] : v[r];
-              v[r] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+              v[r] = keep + __shfl_xor_sync(FULL, send, o);
             }
           } else {
-            v[0] += __shfl_xor_sync(0xffffffffu, v[0], o);
+            v[0] += __shfl_xor_sync(FULL, v[0], o);
           }
         }
-        sv[it] = key < key_lim ? v[0] * scale_log2 : NEG_INF;
+        sv[it] = key < key_lim ? v[0] : NEG_INF;
         wm = fmaxf(wm, sv[it]);
       }
-      // max over this warp's keys for my_row: combine the `sub` lanes
+      // max over the warp's keys for row_q
+      if constexpr (C::kKeyMajor) {
 #pragma unroll
-      for (int o = C::kCPK; o < 32; o <<= 1) wm = fmaxf(wm, __shfl_xor_sync(0xffffffffu, wm, o));
-      if (writer && sub == 0) wmax[((i & 1) * kWarps + warp) * G + my_row] = wm;
+        for (int o = C::kP; o < 32; o <<= 1) wm = fmaxf(wm, __shfl_xor_sync(FULL, wm, o));
+      } else {
+#pragma unroll
+        for (int o = 1; o < C::kKPI; o <<= 1) wm = fmaxf(wm, __shfl_xor_sync(FULL, wm, o));
+      }
+      if (kl == 0 && leader) wmax[((i & 1) * kWarps + warp) * G + row_q] = wm;
     }
     if (__syncthreads_or(!ok)) {  // the single per-tile barrier; also a uniform give-up
       ok = false;
       break;
     }
-    // ---------------- B: decision for tile i (the same in every thread)
+    // ---------------- B: decision for tile i, taken identically by every warp
     bool keep_i = false;
     if (i < nt) {
-      bool all_pass = !tau_is_inf;
+      const float* wb = wmax + (i & 1) * kWarps * G;
+      float mt = lane < n_dec ? wb[lane] : NEG_INF;
+      if constexpr (G == 8) mt = fmaxf(mt, wb[lane + 32]);
 #pragma unroll
-      for (int r = 0; r < G; ++r) {
-        float mt = NEG_INF;
+      for (int o = G; o < n_dec; o <<= 1) mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, o));
+      // row lane % G passes iff it has a history and the tile max is below m - tau
+      const bool pass =
+          lane >= n_dec || (m_exact != NEG_INF && (mt == NEG_INF || mt < m_exact - tau_log2));
+      keep_i = tau_is_inf || !__all_sync(FULL, pass);
+      m_exact = fmaxf(m_exact, mt);  // a skipped tile never raises it
+      if (keep_i) {
+        const bool moved = m_exact > m_ref + kRefSlack;
+        if (__any_sync(FULL, moved)) {
+          const float ref_new = moved ? m_exact : m_ref;
+          const float sc = moved ? ex2(m_ref - ref_new) : 1.f;  // m_ref = -inf gives 0
+          lsum *= __shfl_sync(FULL, sc, row_q);
+          m_ref = ref_new;
+          if (warp == 0 && lane < G) ref_ring[(i % kPRing) * 8 + lane] = ref_new;
+          if (tid == 0) flag_ring[i % kPRing] = 1;
+        } else if (tid == 0) {
+          flag_ring[i % kPRing] = 0;
+        }
+        // probabilities of tile i relative to the reference max of each row
+        const float mr = __shfl_sync(FULL, m_ref, row_q);
+        float* pr = p_ring + (i % kPRing) * kDecodeTile * G;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) mt = fmaxf(mt, wmax[((i & 1) * kWarps + w) * G + r]);
-        const bool pass = m_exact[r] != NEG_INF && (mt == NEG_INF || mt < m_exact[r] - tau_log2);
-        all_pass = all_pass && pass;
-        m_exact[r] = fmaxf(m_exact[r], mt);
+        for (int it = 0; it < C::kSIters; ++it) {
+          const int key = warp * C::kKeysPerWarp + it * C::kKPI + kl;
+          const float p = ex2(sv[it] - mr);
+          if (leader) {
+            pr[key * G + row_q] = p;
+            lsum += p;
+          }
+        }
       }
-      keep_i = !all_pass;
       if (tid == 0) {
         const int t = t_begin + i;
-        if (skip_mask)
-          skip_mask[(static_cast<size_t>(b) * Hkv + kv) * n_tiles_all + t] = keep_i ? 0 : 1;
+        if (skip_mask) skip_mask[static_cast<size_t>(bh) * n_tiles_all + t] = keep_i ? 0 : 1;
         if (keep_i) {  // the slot's previous tile finished its P*V before this barrier
           const int vs = v_issued % kVStages;
-          mbar_arrive_expect_tx(b_v_full(vs), tile_bytes(t));
-          bulk_load(sbase + C::kOffV + vs * C::kTileBytes,
-                    Vg + static_cast<size_t>(t) * kDecodeTile * D, tile_bytes(t), b_v_full(vs));
+          issue(sbase + C::kOffV + vs * C::kTileBytes, &tmV, b_v_full(vs), t);
           ++v_issued;
         }
         if (i + kKStages < nt) {  // every thread has finished reading K slot i % kKStages
           const int ks = i % kKStages;
-          const int tn = t + kKStages;
-          mbar_arrive_expect_tx(b_k_full(ks), tile_bytes(tn));
-          bulk_load(sbase + C::kOffK + ks * C::kTileBytes,
-                    Kg + static_cast<size_t>(tn) * kDecodeTile * D, tile_bytes(tn), b_k_full(ks));
+          issue(sbase + C::kOffK + ks * C::kTileBytes, &tmK, b_k_full(ks), t + kKStages);
           ++k_issued;
         }
       }
-      // probabilities of tile i relative to the running max after tile i
-      if (keep_i && writer) {
-        float* pr = p_ring + (i % kPRing) * kDecodeTile * G;
-        float mr = NEG_INF;
-#pragma unroll
-        for (int r = 0; r < G; ++r)
-          if (r == my_row) mr = m_exact[r];
-#pragma unroll
-        for (int it = 0; it < C::kIters; ++it) {
-          const int key = warp * C::kKeysPerWarp + it * C::kKPI + sub;
-          pr[key * G + my_row] = ex2(sv[it] - mr);
-        }
-      }
     }
-    // shift the per-tile history: running max after tile i, kept bit of tile i
-#pragma unroll
-    for (int k = kLag; k >= 1; --k)
-#pragma unroll
-      for (int r = 0; r < G; ++r) m_hist[k][r] = m_hist[k - 1][r];
-#pragma unroll
-    for (int r = 0; r < G; ++r) m_hist[0][r] = m_exact[r];
     kept_bits = (kept_bits << 1) | (keep_i ? 1u : 0u);
 
     // ---------------- C: P*V of tile t = i - kLag (its p were written kLag barriers ago)
@@ -288,40 +366,35 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
       const bool got = mbar_wait(b_v_full(vs), (pv_count / kVStages) & 1, never, wait_limit_ns);
       ok = ok && got;  // acted on at the next barrier
       if (got) {
-        // move the reference max of the partial sums up to this tile's
+        if (flag_ring[t % kPRing]) {  // move the sums to this tile's reference max
+          float rn[G];
+          load_row_floats<G>(ref_ring + (t % kPRing) * 8, rn);
 #pragma unroll
-        for (int r = 0; r < G; ++r) {
-          const float mn = m_hist[kLag][r];
-          if (mn != m_acc[r]) {
-            const float a = ex2(m_acc[r] - mn);  // m_acc = -inf initially gives 0
-            lsum[r] *= a;
-            const float2 a2 = make_float2(a, a);
+          for (int r = 0; r < G; ++r) {
+            if (rn[r] != m_acc[r]) {
+              const float a = ex2(m_acc[r] - rn[r]);  // m_acc = -inf initially gives 0
+              const float2 a2 = make_float2(a, a);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc[r][e] = __fmul2_rn(acc[r][e], a2);
-            m_acc[r] = mn;
+              for (int e = 0; e < 4; ++e) acc[r][e] = __fmul2_rn(acc[r][e], a2);
+              m_acc[r] = rn[r];
+            }
           }
         }
         const uint8_t* vt = smem + C::kOffV + vs * C::kTileBytes;
         const float* pr = p_ring + (t % kPRing) * kDecodeTile * G;
-        const int key_lim = L - (t_begin + t) * kDecodeTile;
 #pragma unroll
-        for (int it = 0; it < C::kIters; ++it) {
-          const int key = warp * C::kKeysPerWarp + it * C::kKPI + sub;
-          if (key < key_lim) {
-            const uint4 u = *reinterpret_cast<const uint4*>(vt + key * D * 2 + c * 16);
-            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-            float2 vf[4];
+        for (int e2 = 0; e2 < C::kVKeys; ++e2) {
+          const int key = kg + C::kGroups * e2;  // rows past L are zeros with p = 0
+          const uint4 u = *reinterpret_cast<const uint4*>(vt + chunk_off<D>(key, ch));
+          float2 vf[4];
+          bf16x8_to_f32(u, vf);
+          float pv[G];
+          load_row_floats<G>(pr + key * G, pv);
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              vf[e] = make_float2(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xffff0000u));
+          for (int r = 0; r < G; ++r) {
+            const float2 p2 = make_float2(pv[r], pv[r]);
 #pragma unroll
-            for (int r = 0; r < G; ++r) {
-              const float pv = pr[key * G + r];
-              const float2 p2 = make_float2(pv, pv);
-#pragma unroll
-              for (int e = 0; e < 4; ++e) acc[r][e] = __ffma2_rn(p2, vf[e], acc[r][e]);
-              if (c == 0) lsum[r] += pv;
-            }
+            for (int e = 0; e < 4; ++e) acc[r][e] = __ffma2_rn(p2, vf[e], acc[r][e]);
           }
         }
       }
@@ -344,56 +417,60 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
     return;
   }
 
-  // ---------------- reduce the partial sums: lanes of one chunk, then warps
+  // ---------------- combine the key subsets: lanes of one warp, then warps
 #pragma unroll
-  for (int o = C::kCPK; o < 32; o <<= 1) {
-#pragma unroll
-    for (int r = 0; r < G; ++r) {
-      lsum[r] += __shfl_xor_sync(0xffffffffu, lsum[r], o);
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        acc[r][e].x += __shfl_xor_sync(0xffffffffu, acc[r][e].x, o);
-        acc[r][e].y += __shfl_xor_sync(0xffffffffu, acc[r][e].y, o);
-      }
-    }
-  }
-  float* red = reinterpret_cast<float*>(smem + C::kOffK);  // [warp][G][D+1]
-  __syncthreads();
-  if (sub == 0) {
+  for (int o = C::kChunks; o < 32; o <<= 1) {
 #pragma unroll
     for (int r = 0; r < G; ++r) {
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        red[(warp * G + r) * (D + 1) + c * 8 + 2 * e] = acc[r][e].x;
-        red[(warp * G + r) * (D + 1) + c * 8 + 2 * e + 1] = acc[r][e].y;
+        acc[r][e].x += __shfl_xor_sync(FULL, acc[r][e].x, o);
+        acc[r][e].y += __shfl_xor_sync(FULL, acc[r][e].y, o);
       }
-      if (c == 0) red[(warp * G + r) * (D + 1) + D] = lsum[r];
     }
   }
-  __syncthreads();
-  for (int idx = tid; idx < G * (D + 1); idx += kDecThreads) {
-    const int r = idx / (D + 1), col = idx % (D + 1);
-    float s = 0.f;
+  float lrow[G];  // sum of p over the warp's keys, per row
 #pragma unroll
-    for (int w = 0; w < kWarps; ++w) s += red[(w * G + r) * (D + 1) + col];
-    red[r * (D + 1) + col] = s;  // warp 0's slot; only this thread touches (r, col)
+  for (int r = 0; r < G; ++r) {
+    float x = row_q == r ? lsum : 0.f;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) x += __shfl_xor_sync(FULL, x, o);
+    lrow[r] = x;
+  }
+  // every copy has landed and been read: the K ring is free for the reduction
+  float* red = reinterpret_cast<float*>(smem + C::kOffK);  // [warp][G][D]
+  if (lane < C::kChunks) {
+#pragma unroll
+    for (int r = 0; r < G; ++r) {
+      float4* dst = reinterpret_cast<float4*>(red + (warp * G + r) * D + ch * 8);
+      dst[0] = make_float4(acc[r][0].x, acc[r][0].y, acc[r][1].x, acc[r][1].y);
+      dst[1] = make_float4(acc[r][2].x, acc[r][2].y, acc[r][3].x, acc[r][3].y);
+    }
+  }
+  if (lane == 0) {
+#pragma unroll
+    for (int r = 0; r < G; ++r) wl[warp * G + r] = lrow[r];
   }
   __syncthreads();
   for (int idx = tid; idx < G * D; idx += kDecThreads) {
     const int r = idx / D, col = idx % D;
+    float s = 0.f, den = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      s += red[(w * G + r) * D + col];
+      den += wl[w * G + r];
+    }
     const size_t row = static_cast<size_t>(b) * Hq + kv * G + r;
-    o_part[(row * n_splits + split) * D + col] = red[r * (D + 1) + col] / red[r * (D + 1) + D];
+    o_part[(row * n_splits + split) * D + col] = s / den;
   }
   if (tid < G) {
-    // every thread holds the same reference max (skipped tiles never move the
-    // running max, so it is the value used by the last P*V); select it with a
-    // constant index
-    float mr = NEG_INF;
+    // lane tid of warp 0 holds the reference max of row tid, which is the one
+    // both the sums of p and the P*V sums are relative to
+    float den = 0.f;
 #pragma unroll
-    for (int r = 0; r < G; ++r)
-      if (r == tid) mr = m_acc[r];
+    for (int w = 0; w < kWarps; ++w) den += wl[w * G + tid];
     const size_t row = static_cast<size_t>(b) * Hq + kv * G + tid;
-    lse_part[row * n_splits + split] = mr + __log2f(red[tid * (D + 1) + D]);
+    lse_part[row * n_splits + split] = m_ref + __log2f(den);
   }
 }
 
@@ -418,6 +495,35 @@ __global__ void __launch_bounds__(D)
 
 namespace {
 
+PFN_cuTensorMapEncodeTiled_v12000 dec_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult qr;
+    void* p = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &qr) == cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// [B*Hkv, L, D] bf16, d fastest; box = 64 columns x 64 keys, 128-byte swizzle,
+// out-of-range keys read as zeros
+bool dec_map(CUtensorMap* m, const void* base, int BH, int L, int D) {
+  auto enc = dec_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(L),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(L) * D * 2};
+  cuuint32_t box[3] = {64, static_cast<cuuint32_t>(kDecodeTile), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D, int G>
 int launch_dg(const DecodeLaunch& a) {
   using C = DecCfg<D, G>;
@@ -431,12 +537,14 @@ int launch_dg(const DecodeLaunch& a) {
       return ATTN_ERR_CUDA;
     attr_done |= uint64_t(1) << dev;
   }
+  CUtensorMap mk, mv;
+  if (!dec_map(&mk, a.K, a.B * a.Hkv, a.L, D) || !dec_map(&mv, a.V, a.B * a.Hkv, a.L, D))
+    return ATTN_ERR_CUDA;
   dim3 grid(a.n_splits, a.Hkv, a.B);
   kern<<<grid, kDecThreads, C::kSmemBytes, a.stream>>>(
-      static_cast<const __nv_bfloat16*>(a.q), static_cast<const __nv_bfloat16*>(a.K),
-      static_cast<const __nv_bfloat16*>(a.V), a.o_part, a.lse_part, a.skip_mask, a.status, a.Hq,
-      a.Hkv, a.L, a.split_len, a.n_splits, a.scale_log2, a.tau_log2, a.tau_is_inf,
-      a.wait_limit_ns);
+      mk, mv, static_cast<const __nv_bfloat16*>(a.q), a.o_part, a.lse_part, a.skip_mask,
+      a.status, a.Hq, a.Hkv, a.L, a.split_len, a.n_splits, a.scale_log2, a.tau_log2,
+      a.tau_is_inf, a.wait_limit_ns);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   decode_combine_kernel<D><<<a.B * a.Hq, D, 0, a.stream>>>(
       a.o_part, a.lse_part, static_cast<__nv_bfloat16*>(a.o), a.n_splits);
