@@ -344,10 +344,10 @@ def main():
     achieved = flops / (ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                 "frac": achieved / peaks["bf16_tflops"],
-                "traffic": measured_traffic("prefill_kernel", "prefill_sm100.cu"),
+                "traffic": measured_traffic("prefill_pp_kernel", "prefill_pp_sm100.cu"),
                 "algorithmic_bytes": compulsory_prefill_bytes(w),
                 "peak_source": f"{peak_src} bf16 burst (kernel timed alone)",
-                "kernel": "prefill_kernel<128,128,64,false>",
+                "kernel": "prefill_pp_kernel<128,64,false> (two 128-row blocks per CTA, persistent)",
                 "algorithmic": "4*B*Hq*N^2*d dense-equivalent FLOPs per launch"}
     clk = clocks.summary(t0, t1) if rank == 0 else None
 
