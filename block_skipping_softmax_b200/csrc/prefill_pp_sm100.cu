@@ -35,6 +35,7 @@
 
 #include <cstdint>
 
+#include "exp2_poly.cuh"
 #include "kernels.cuh"
 #include "ptx.cuh"
 
@@ -48,6 +49,14 @@ constexpr int kRows = 128;    // rows per tile (row block)
 constexpr int kDR = 4;        // decision ring
 constexpr int kCR = 16;       // commit ring per row block (waiters lag by at most ~6)
 constexpr float kRescale = 8.0f;  // lazy rescale threshold (log2 units)
+// Which of the 16 column pairs of each 32-column chunk take the polynomial
+// exp2 instead of MUFU (bit c = pair c).  Measured on B200 the softmax here is
+// not bound by MUFU throughput, and every fraction tried (1/4 to 3/4) made
+// the kernel slower, so the default is none.
+#ifndef BSS_POLY_PAIRS
+#define BSS_POLY_PAIRS 0x0000u
+#endif
+constexpr uint32_t kPolyPairs = BSS_POLY_PAIRS;
 
 template <int D, int BC>
 struct PPCfg {
@@ -89,6 +98,7 @@ struct PPMisc {
   int abort;
   int dec[2][kDR];
   int vote[2][2][4];
+  int leave[2][4];
 };
 
 __device__ __forceinline__ void named_bar(int id, int count) {
@@ -582,11 +592,13 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           m_ref = m_cand;
         }
         // P = 2^(s*scale - m_ref): one packed FFMA per pair, two ex2, one
-        // pack; the row sum adds the bf16-rounded pair with one packed add
+        // pack to bf16 for the P*V MMA; the row sum adds the fp32 pair with
+        // one packed add (four independent chains)
         const float neg_m = row_valid ? -m_ref : 0.f;  // invalid rows: all scores -inf -> P = 0
         const float2 sc2 = make_float2(scale_log2, scale_log2);
         const float2 nm2 = make_float2(neg_m, neg_m);
-        float2 rs2 = make_float2(0.f, 0.f);
+        float2 rs2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                         make_float2(0.f, 0.f)};  // four independent add chains
 #pragma unroll
         for (int c0 = 0; c0 < BC; c0 += 32) {
           uint32_t pk[16];
@@ -595,13 +607,23 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             const float2 x = __ffma2_rn(
                 make_float2(__uint_as_float(u[c0 + 2 * c]), __uint_as_float(u[c0 + 2 * c + 1])), sc2,
                 nm2);
-            const uint32_t w = pack_bf16x2(ex2(x.x), ex2(x.y));
-            rs2 = __fadd2_rn(rs2, make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u)));
+            // pairs in kPolyPairs take 2^x on the FMA pipes, the rest on MUFU
+            uint32_t w;
+            if ((kPolyPairs >> c) & 1u) {  // 2^x on the FMA pipes; the sum takes the bf16 values
+              w = exp2_poly_bf16x2(x);
+              rs2[c & 3] = __fadd2_rn(rs2[c & 3], make_float2(__uint_as_float(w << 16),
+                                                              __uint_as_float(w & 0xffff0000u)));
+            } else {  // 2^x on MUFU; the sum takes the fp32 values
+              const float2 e = make_float2(ex2(x.x), ex2(x.y));
+              w = pack_bf16x2(e.x, e.y);
+              rs2[c & 3] = __fadd2_rn(rs2[c & 3], e);
+            }
             pk[c] = w;
           }
           tmem_st16(tS(t, sb) + lane_off + c0 / 2, pk);
         }
-        l_sum = l_sum * alpha + (rs2.x + rs2.y);
+        const float2 rsa = __fadd2_rn(__fadd2_rn(rs2[0], rs2[1]), __fadd2_rn(rs2[2], rs2[3]));
+        l_sum = l_sum * alpha + (rsa.x + rsa.y);
         // O rescale (after the P store, so the scores are no longer live).
         // P*V of tile j-1 must have finished: commit #(base + pro + j - 1).
         // With one S buffer that is the commit S_j already waited for.
@@ -633,14 +655,26 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           break;
         }
       }
-      if (failed) ok = false;
+      // Leaving the loop above is collective for the four warps of this row
+      // block (after a vote, or per warp only with tau = inf, where they
+      // never meet at a named barrier).  A give-up recorded after the last
+      // vote, and the wait for the last P*V below, can differ between warps:
+      // with a finite tau they are combined here, so that no warp goes on to
+      // the next item's votes while another has left.
       if (!ok) break;
       // ---- epilogue: O / l -> bf16 -> global; unvisited tiles marked 2
       if (skip_mask)
         for (int j = T + row; j < n_tiles; j += 128) skip_mask[mask_base + j] = 2;
       // P*V of the last tile finished: commit #(base + pro + T - 1)
-      const bool done = __all_sync(0xffffffffu, wait_cm(t, base + pro + T - 1));
+      bool done = !failed && __all_sync(0xffffffffu, wait_cm(t, base + pro + T - 1));
       base += pro + T;
+      if (!tau_is_inf) {
+        if (lane == 0) reinterpret_cast<volatile int*>(misc->leave[t])[sw] = done ? 0 : 1;
+        named_bar(1 + t, 128);
+#pragma unroll
+        for (int w = 0; w < 4; ++w)
+          if (reinterpret_cast<volatile int*>(misc->leave[t])[w]) done = false;
+      }
       if (!done) {
         pp_give_up(misc, status, 11);
         ok = false;
