@@ -73,6 +73,9 @@ struct PPCfg {
   // Q slots: with two, the next work item's Q loads while this one runs
   static constexpr int kQS = (BC == 128 && D == 128) ? 1 : 2;
   static constexpr int kQSlot = 2 * kQTile;  // two row blocks
+  // With two Q slots, a row block's O is staged in its own (finished) Q tile
+  // and written by a TMA store; the slot is released once the store has read it.
+  static constexpr bool kTmaEpi = kQS == 2;
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQS * kQSlot;
   static constexpr int kOffV = kOffK + kKS * kKVBytes;
@@ -98,7 +101,7 @@ struct PPMisc {
   int abort;
   int dec[2][kDR];
   int vote[2][2][4];
-  int leave[2][4];
+  int leave[2][2][4];
 };
 
 __device__ __forceinline__ void named_bar(int id, int count) {
@@ -177,7 +180,8 @@ struct Pending3 {
 template <int D, int BC, bool CAUSAL>
 __global__ void __launch_bounds__(kPPThreads, 1)
     prefill_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                      const __grid_constant__ CUtensorMap tmV, __nv_bfloat16* __restrict__ O,
+                      const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
+                      __nv_bfloat16* __restrict__ O,
                       uint8_t* __restrict__ skip_mask, int* __restrict__ status, int B, int Hq,
                       int Hkv, int N, float scale_log2, float tau_log2, int tau_is_inf,
                       unsigned long long wait_limit_ns) {
@@ -230,7 +234,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
     }
     for (int s = 0; s < C::kQS; ++s) {
       mbar_init(b_q_full(s), 1);
-      mbar_init(b_q_empty(s), 1);
+      mbar_init(b_q_empty(s), C::kTmaEpi ? 2 : 1);  // one arrival per row block's O store
     }
     mbar_init(b_mma_done, 1);
     misc->abort = 0;
@@ -429,7 +433,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         }
         if (!alive) break;
         // the Q slot is free once the item's last S MMA has run
-        if (it.Tmax <= SB) mma_commit(b_q_empty(qs));
+        if (!C::kTmaEpi && it.Tmax <= SB) mma_commit(b_q_empty(qs));
         bool started[2] = {false, false};
         for (int j = 0; alive && j < it.Tmax; ++j) {
           bool v_used = false, k_next = false;
@@ -483,7 +487,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           }
           if (k_next) ++kuse;
           if (v_used) ++vuse;
-          if (j + SB + 1 == it.Tmax) mma_commit(b_q_empty(qs));  // last S MMAs issued
+          if (!C::kTmaEpi && j + SB + 1 == it.Tmax) mma_commit(b_q_empty(qs));  // last S MMAs issued
         }
       }
       // all issued MMAs must finish before TMEM is released
@@ -499,12 +503,29 @@ __global__ void __launch_bounds__(kPPThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(sw * 32) << 16;
     const float NEG_INF = -__int_as_float(0x7f800000);
     int sc = 0, dcount = 0;
-    int base = 0;  // this row block's commits in earlier items
+    int base = 0;    // this row block's commits in earlier items
+    int items = 0;   // work items seen (the Q slot of item i is i % kQS)
+    int leaves = 0;  // item-end synchronisations of this warpgroup
+    // thread 0 of the warpgroup: the Q slot its last O store reads, and how
+    // many arrivals on that slot's q_empty the store stands for
+    int pend_slot = -1, pend_n = 0;
+    auto release_pending = [&]() {
+      if (C::kTmaEpi && pend_slot >= 0) {
+        bulk_wait_read_all();
+        for (int k = 0; k < pend_n; ++k) mbar_arrive(b_q_empty(pend_slot));
+        pend_slot = -1;
+      }
+    };
     bool ok = true, failed = false;
     for (long long idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
       const Item it = make_item<BC, CAUSAL>(idx, BH, n_pairs, n_rb, N);
       const int T = t == 0 ? it.T0 : it.T1;
-      if (T == 0) continue;  // this row block does not exist
+      const int qs = items % C::kQS;
+      ++items;
+      if (T == 0) {  // this row block does not exist
+        release_pending();
+        continue;
+      }
       const int pro = min(SB, T);
       const int rb = it.rb0 + t;
       const int q_idx = rb * kRows + row;
@@ -566,9 +587,12 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           if (bad) waited = false;
         }
         if (!waited) {
-          pp_give_up(misc, status, 10);
-          ok = false;
-          break;
+          // With a finite tau the vote made this branch common to the four
+          // warps; with tau = inf no warp meets the others inside the loop.
+          // Either way the warps run out the item and leave together below.
+          if (!failed) pp_give_up(misc, status, 10);
+          failed = true;
+          continue;
         }
         m_exact = fmaxf(m_exact, mt);
         const int di = dcount % kDR;
@@ -581,6 +605,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         if (skip) {
           __syncwarp();
           if (lane == 0) mbar_arrive(b_p_full(t, sb));
+          if (j == 0) release_pending();
           continue;
         }
         // ---- kept tile: lazy reference max, P, then O rescale
@@ -650,58 +675,93 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(b_p_full(t, sb));
-        if (failed && tau_is_inf) {  // no votes without a finite tau: stop here
-          ok = false;
-          break;
-        }
+        // the previous item's O store has had a tile's time to read its Q slot
+        if (j == 0) release_pending();
       }
-      // Leaving the loop above is collective for the four warps of this row
-      // block (after a vote, or per warp only with tau = inf, where they
-      // never meet at a named barrier).  A give-up recorded after the last
-      // vote, and the wait for the last P*V below, can differ between warps:
-      // with a finite tau they are combined here, so that no warp goes on to
-      // the next item's votes while another has left.
-      if (!ok) break;
       // ---- epilogue: O / l -> bf16 -> global; unvisited tiles marked 2
       if (skip_mask)
         for (int j = T + row; j < n_tiles; j += 128) skip_mask[mask_base + j] = 2;
-      // P*V of the last tile finished: commit #(base + pro + T - 1)
+      // P*V of the last tile finished: commit #(base + pro + T - 1).  A give-up
+      // (recorded by any warp during the item) or a failed wait is combined
+      // over the four warps, which then go on, or leave, together.
       bool done = !failed && __all_sync(0xffffffffu, wait_cm(t, base + pro + T - 1));
       base += pro + T;
-      if (!tau_is_inf) {
-        if (lane == 0) reinterpret_cast<volatile int*>(misc->leave[t])[sw] = done ? 0 : 1;
+      {
+        volatile int* lv = misc->leave[t][leaves & 1];
+        ++leaves;
+        if (lane == 0) lv[sw] = done ? 0 : 1;
         named_bar(1 + t, 128);
 #pragma unroll
         for (int w = 0; w < 4; ++w)
-          if (reinterpret_cast<volatile int*>(misc->leave[t])[w]) done = false;
+          if (lv[w]) done = false;
       }
       if (!done) {
-        pp_give_up(misc, status, 11);
+        if (!failed) pp_give_up(misc, status, 11);
         ok = false;
         break;
       }
       tc_fence_after();
       const float inv_l = row_valid ? 1.f / l_sum : 0.f;
-      __nv_bfloat16* orow = O + (static_cast<size_t>(it.bh) * N + (row_valid ? q_idx : 0)) * D;
+      if constexpr (C::kTmaEpi) {
+        // Stage O (bf16) in this row block's Q tile, which no MMA reads any
+        // more (its last S MMA completed before the last P*V), in the TMA
+        // layout (64-column panels, 128-byte swizzle), then one thread stores
+        // the tile; rows past N are clipped by the store.
+        const uint32_t stage = sQ + qs * C::kQSlot + t * C::kQTile;
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t r[32];
-        tmem_ld32(tO(t) + lane_off + c0, r);
-        tmem_wait_ld();
-        if (row_valid) {
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(tO(t) + lane_off + c0, r);
+          tmem_wait_ld();
           uint32_t w[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c)
             w[c] = pack_bf16x2(__uint_as_float(r[2 * c]) * inv_l, __uint_as_float(r[2 * c + 1]) * inv_l);
-          uint4* dst = reinterpret_cast<uint4*>(orow + c0);
 #pragma unroll
-          for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+          for (int q = 0; q < 4; ++q) {
+            const int lc = c0 / 8 + q;  // 16-byte chunk of the row
+            const uint32_t a = stage + (lc >> 3) * C::kQPanel + row * 128 + (((lc & 7) ^ (row & 7)) << 4);
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(w[4 * q]),
+                         "r"(w[4 * q + 1]), "r"(w[4 * q + 2]), "r"(w[4 * q + 3])
+                         : "memory");
+          }
+        }
+        fence_proxy_async_smem();  // the generic-proxy writes, before the async-proxy store
+        named_bar(1 + t, 128);
+        if (row == 0) {
+          release_pending();  // at most one store in flight per warpgroup
+#pragma unroll
+          for (int p = 0; p < C::kPanels; ++p)
+            tma_store_3d(&tmO, stage + p * C::kQPanel, p * 64, rb * kRows, it.bh);
+          bulk_commit_group();
+          pend_slot = qs;
+          pend_n = (t == 0 && it.T1 == 0) ? 2 : 1;  // row block 1 absent: arrive for it too
+        }
+      } else {
+        __nv_bfloat16* orow = O + (static_cast<size_t>(it.bh) * N + (row_valid ? q_idx : 0)) * D;
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(tO(t) + lane_off + c0, r);
+          tmem_wait_ld();
+          if (row_valid) {
+            uint32_t w[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+              w[c] = pack_bf16x2(__uint_as_float(r[2 * c]) * inv_l, __uint_as_float(r[2 * c + 1]) * inv_l);
+            uint4* dst = reinterpret_cast<uint4*>(orow + c0);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+          }
         }
       }
       // O_t may be overwritten by the next item's first P*V only after this
       // warpgroup signals that item's first P: ordering comes from p_full.
       tc_fence_before();
     }
+    // no store may still be reading shared memory, or writing O, at exit
+    release_pending();
+    if (C::kTmaEpi && row == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -762,15 +822,15 @@ int pp_launch(const PrefillLaunch& a) {
       return ATTN_ERR_CUDA;
     ready |= uint64_t(1) << dev;
   }
-  CUtensorMap mq, mk, mv;
+  CUtensorMap mq, mk, mv, mo;
   if (!pp_map(&mq, a.Q, a.B * a.Hq, a.N, D, kRows) || !pp_map(&mk, a.K, a.B * a.Hkv, a.N, D, BC) ||
-      !pp_map(&mv, a.V, a.B * a.Hkv, a.N, D, BC))
+      !pp_map(&mv, a.V, a.B * a.Hkv, a.N, D, BC) || !pp_map(&mo, a.O, a.B * a.Hq, a.N, D, kRows))
     return ATTN_ERR_CUDA;
   const long long n_rb = (a.N + kRows - 1) / kRows;
   const long long n_items = static_cast<long long>(a.B) * a.Hq * ((n_rb + 1) / 2);
   const int grid = static_cast<int>(n_items < sm_count[dev] ? n_items : sm_count[dev]);
   kern<<<grid, kPPThreads, C::kSmemBytes, a.stream>>>(
-      mq, mk, mv, static_cast<__nv_bfloat16*>(a.O), a.skip_mask, a.status, a.B, a.Hq, a.Hkv, a.N,
+      mq, mk, mv, mo, static_cast<__nv_bfloat16*>(a.O), a.skip_mask, a.status, a.B, a.Hq, a.Hkv, a.N,
       a.scale_log2, a.tau_log2, a.tau_is_inf, a.wait_limit_ns);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
