@@ -99,8 +99,11 @@ struct PPCfg {
 struct PPMisc {
   uint32_t tmem_base;
   int abort;
-  int dec[2][kDR];
-  int vote[2][2][4];
+  // vote[t][i][w]: (decision number << 2) | 2 if warp w of row block t gave
+  // up | 1 if every row of that warp passes the skip test, for the decision
+  // in ring slot i (the decision number runs over all key tiles a row block
+  // visits).  The tile is skipped iff all four warps pass.
+  int vote[2][kDR][4];
   int leave[2][2][4];
 };
 
@@ -209,7 +212,11 @@ __global__ void __launch_bounds__(kPPThreads, 1)
   const uint32_t b_mma_done = bar0 + 8u * (kBQ + 2 * C::kQS);
   PPMisc* misc = reinterpret_cast<PPMisc*>(smem + C::kOffMisc);
   volatile int* abort_flag = &misc->abort;
-  volatile int* vdec = &misc->dec[0][0];
+  // keep (1) or skip (0) from the four vote words of one decision
+  auto decided_keep = [&](int t, int i) -> int {
+    const volatile int* v = misc->vote[t][i];
+    return ((v[0] & v[1] & v[2] & v[3]) & 1) ? 0 : 1;
+  };
   // wait for commit number i of row block t (bounded)
   auto wait_cm = [&](int t, int i) {
     return mbar_wait(b_cm(t, i), (i / kCR) & 1, abort_flag, wait_limit_ns);
@@ -230,13 +237,16 @@ __global__ void __launch_bounds__(kPPThreads, 1)
     for (int t = 0; t < 2; ++t) {
       for (int i = 0; i < kCR; ++i) mbar_init(b_cm(t, i), 1);
       for (int b = 0; b < SB; ++b) mbar_init(b_p_full(t, b), 4);
-      for (int i = 0; i < kDR; ++i) mbar_init(b_dec(t, i), 1);
+      for (int i = 0; i < kDR; ++i) mbar_init(b_dec(t, i), 4);  // one arrival per softmax warp
     }
     for (int s = 0; s < C::kQS; ++s) {
       mbar_init(b_q_full(s), 1);
       mbar_init(b_q_empty(s), C::kTmaEpi ? 2 : 1);  // one arrival per row block's O store
     }
     mbar_init(b_mma_done, 1);
+    for (int t = 0; t < 2; ++t)
+      for (int i = 0; i < kDR; ++i)
+        for (int w = 0; w < 4; ++w) misc->vote[t][i][w] = -1;  // no decision number matches
     misc->abort = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -361,7 +371,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
               continue;
             }
             ++dl[t];
-            if (vdec[t * kDR + di] && !issued) {
+            if (decided_keep(t, di) && !issued) {
               if (!issue_v(j)) {
                 pp_give_up(misc, status, 4);
                 alive = false;
@@ -448,7 +458,8 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             }
             ++pc[t];
             tc_fence_after();
-            const int keep = vdec[t * kDR + (dc[t] % kDR)];
+            // every warp wrote its vote before arriving on p_full
+            const int keep = tau_is_inf ? 1 : decided_keep(t, dc[t] % kDR);
             ++dc[t];
             if (keep) {
               if (!v_used) {
@@ -564,44 +575,60 @@ __global__ void __launch_bounds__(kPPThreads, 1)
               m4[k] = fmax3(m4[k], __uint_as_float(u[c + 2 * k]), __uint_as_float(u[c + 2 * k + 1]));
           mt = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * scale_log2;  // log2 units; -inf stays -inf
         }
-        // ---- skip test: every row of this row block must have mt < m - tau
+        // ---- skip test: every row of this row block must have mt < m - tau.
+        // Each warp publishes its own verdict (all its rows pass, or not) and
+        // arrives on the decision barrier.  A warp with a row that fails knows
+        // at once that the tile is kept; only a warp whose rows all pass looks
+        // at the other three verdicts, and stops at the first that fails.
+        const int di = dcount % kDR;
+        const int dnum = dcount;
+        ++dcount;
         bool skip = false;
-        if (!tau_is_inf) {
-          const bool pass =
-              !row_valid || (m_exact != NEG_INF && (mt == NEG_INF || mt < m_exact - tau_log2));
-          const unsigned all_pass = __all_sync(0xffffffffu, pass);
-          const unsigned all_ok = __all_sync(0xffffffffu, waited);
-          const int slot = j & 1;
-          if (lane == 0)
-            reinterpret_cast<volatile int*>(misc->vote[t][slot])[sw] =
-                (all_pass ? 1 : 0) | (all_ok ? 0 : 2);
-          named_bar(1 + t, 128);
-          int v = 1, bad = 0;
-#pragma unroll
-          for (int w = 0; w < 4; ++w) {
-            const int vw = reinterpret_cast<volatile int*>(misc->vote[t][slot])[w];
-            v &= vw & 1;
-            bad |= vw & 2;
+        if (!tau_is_inf) {  // with tau = inf every tile is kept and nobody reads votes
+          const bool pass = waited &&
+                            (!row_valid || (m_exact != NEG_INF && (mt == NEG_INF || mt < m_exact - tau_log2)));
+          const bool warp_pass = __all_sync(0xffffffffu, pass) != 0;
+          const bool warp_ok = __all_sync(0xffffffffu, waited) != 0;
+          volatile int* vv = misc->vote[t][di];
+          if (lane == 0) {
+            vv[sw] = (dnum << 2) | (warp_ok ? 0 : 2) | (warp_pass ? 1 : 0);
+            mbar_arrive(b_dec(t, di));
           }
-          skip = v != 0;
-          if (bad) waited = false;
+          if (warp_pass) {
+            int verdict = 0;  // 1 keep, 2 skip, 3 gave up
+            if (lane == 0) {
+              const uint64_t t0 = globaltimer_ns();
+              for (uint32_t n = 0; verdict == 0; ++n) {
+                int n_pass = 0;
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                  const int x = vv[w];
+                  if ((x >> 2) == dnum) {
+                    if (x & 1) ++n_pass;
+                    else verdict = 1;
+                  }
+                }
+                if (verdict == 0 && n_pass == 4) verdict = 2;
+                if (verdict == 0 && (n & 15u) == 15u &&
+                    (*abort_flag || globaltimer_ns() - t0 > wait_limit_ns))
+                  verdict = 3;
+                if (verdict == 0 && n >= 2) __nanosleep(64);  // leave the issue slots to the others
+              }
+            }
+            verdict = __shfl_sync(0xffffffffu, verdict, 0);
+            if (verdict == 3) waited = false;
+            skip = verdict == 2;
+          }
         }
         if (!waited) {
-          // With a finite tau the vote made this branch common to the four
-          // warps; with tau = inf no warp meets the others inside the loop.
-          // Either way the warps run out the item and leave together below.
+          // The warps of this row block run out the item and leave together
+          // at the item-end synchronisation below.
           if (!failed) pp_give_up(misc, status, 10);
           failed = true;
           continue;
         }
         m_exact = fmaxf(m_exact, mt);
-        const int di = dcount % kDR;
-        ++dcount;
-        if (row == 0) {
-          vdec[t * kDR + di] = skip ? 0 : 1;
-          if (skip_mask) skip_mask[mask_base + j] = skip ? 1 : 0;
-          mbar_arrive(b_dec(t, di));
-        }
+        if (row == 0 && skip_mask) skip_mask[mask_base + j] = skip ? 1 : 0;
         if (skip) {
           __syncwarp();
           if (lane == 0) mbar_arrive(b_p_full(t, sb));
