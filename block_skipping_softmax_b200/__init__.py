@@ -22,7 +22,7 @@ __all__ = [
     "attn_decode_noalloc",
     "attn_decode_split_len", "attn_decode_tile", "attn_decode_workspace_bytes",
     "attn_set_stream", "attn_sync_status", "attn_last_timeout_site", "attn_set_wait_limit_ms",
-    "attn_status_string", "attn_shutdown", "prefill", "decode", "STATUS",
+    "attn_test_withhold_copy", "attn_status_string", "attn_shutdown", "prefill", "decode", "STATUS",
 ]
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -62,6 +62,7 @@ def lib() -> ctypes.CDLL:
         "attn_sync_status": (ci, []),
         "attn_last_timeout_site": (ci, []),
         "attn_set_wait_limit_ms": (ci, [ci]),
+        "attn_test_withhold_copy": (ci, [ci]),
         "attn_status_string": (ctypes.c_char_p, [ci]),
         "attn_shutdown": (None, []),
     }
@@ -122,6 +123,11 @@ def attn_last_timeout_site() -> int:
 
 def attn_set_wait_limit_ms(ms) -> int:
     return lib().attn_set_wait_limit_ms(int(ms))
+
+
+def attn_test_withhold_copy(which) -> int:
+    """Test support: 1 = decode CTAs withhold their first V copy (the waits run out)."""
+    return lib().attn_test_withhold_copy(int(which))
 
 
 def attn_status_string(status) -> str:

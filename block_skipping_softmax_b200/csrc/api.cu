@@ -21,6 +21,7 @@ std::mutex g_mu;
 cudaStream_t g_stream = nullptr;
 unsigned long long g_wait_limit_ns = 2000ull * 1000ull * 1000ull;
 int g_last_site = 0;
+int g_withhold_v = 0;  // test support, see attn_test_withhold_copy
 int g_dev_checked[kMaxDevices];  // 0 unknown, 1 sm_100, 2 other
 int* g_status_ptr[kMaxDevices];
 void* g_ws[kMaxDevices];
@@ -226,6 +227,10 @@ int attn_decode_ex(const void* q, const void* K, const void* V, void* o, int B, 
   a.status = status;
   a.wait_limit_ns = g_wait_limit_ns;
   a.stream = static_cast<cudaStream_t>(stream);
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    a.withhold_v = g_withhold_v;
+  }
   return bss::launch_decode(a);
 }
 
@@ -244,6 +249,13 @@ int attn_set_wait_limit_ms(int ms) {
   if (ms < 1) return ATTN_ERR_INVALID_ARG;
   std::lock_guard<std::mutex> lk(g_mu);
   g_wait_limit_ns = static_cast<unsigned long long>(ms) * 1000000ull;
+  return ATTN_OK;
+}
+
+int attn_test_withhold_copy(int which) {
+  if (which != 0 && which != 1) return ATTN_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lk(g_mu);
+  g_withhold_v = which;
   return ATTN_OK;
 }
 

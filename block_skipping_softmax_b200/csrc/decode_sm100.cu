@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
                           float* __restrict__ lse_part, uint8_t* __restrict__ skip_mask,
                           int* __restrict__ status, int Hq, int Hkv, int L, int split_len,
                           int n_splits, float scale_log2, float tau_log2, int tau_is_inf,
-                          unsigned long long wait_limit_ns) {
+                          unsigned long long wait_limit_ns, int withhold_v) {
   using C = DecCfg<D, G>;
   constexpr unsigned FULL = 0xffffffffu;
   constexpr int kLog2P = ilog2(C::kP);
@@ -347,7 +347,10 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
         if (skip_mask) skip_mask[static_cast<size_t>(bh) * n_tiles_all + t] = keep_i ? 0 : 1;
         if (keep_i) {  // the slot's previous tile finished its P*V before this barrier
           const int vs = v_issued % kVStages;
-          issue(sbase + C::kOffV + vs * C::kTileBytes, &tmV, b_v_full(vs), t);
+          // test support: the first copy can be withheld, so that every wait
+          // for it runs out and the timeout path is exercised
+          if (!(withhold_v && v_issued == 0))
+            issue(sbase + C::kOffV + vs * C::kTileBytes, &tmV, b_v_full(vs), t);
           ++v_issued;
         }
         if (i + kKStages < nt) {  // every thread has finished reading K slot i % kKStages
@@ -412,7 +415,8 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
       for (int k = max(0, k_issued - kKStages); k < k_issued; ++k)
         mbar_drain(b_k_full(k % kKStages), (k / kKStages) & 1, wait_limit_ns);
       for (int k = max(0, v_issued - kVStages); k < v_issued; ++k)
-        mbar_drain(b_v_full(k % kVStages), (k / kVStages) & 1, wait_limit_ns);
+        if (!(withhold_v && k == 0))  // a withheld copy was never issued
+          mbar_drain(b_v_full(k % kVStages), (k / kVStages) & 1, wait_limit_ns);
     }
     return;
   }
@@ -544,7 +548,7 @@ int launch_dg(const DecodeLaunch& a) {
   kern<<<grid, kDecThreads, C::kSmemBytes, a.stream>>>(
       mk, mv, static_cast<const __nv_bfloat16*>(a.q), a.o_part, a.lse_part, a.skip_mask,
       a.status, a.Hq, a.Hkv, a.L, a.split_len, a.n_splits, a.scale_log2, a.tau_log2,
-      a.tau_is_inf, a.wait_limit_ns);
+      a.tau_is_inf, a.wait_limit_ns, a.withhold_v);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   decode_combine_kernel<D><<<a.B * a.Hq, D, 0, a.stream>>>(
       a.o_part, a.lse_part, static_cast<__nv_bfloat16*>(a.o), a.n_splits);

@@ -47,6 +47,7 @@ struct DecodeLaunch {
   int* status;
   unsigned long long wait_limit_ns;
   cudaStream_t stream;
+  int withhold_v;  // test support: 1 = every CTA withholds its first V copy
 };
 
 int launch_decode(const DecodeLaunch& a);

@@ -153,6 +153,17 @@ ATTN_API int attn_last_timeout_site(void);
  * (default 2000).  Values < 1 are rejected. */
 ATTN_API int attn_set_wait_limit_ms(int ms);
 
+/* Test support for the timeout path (no fault, trap or hang is involved).
+ * which = 1: every CTA of the following attn_decode / attn_decode_ex calls
+ * withholds the copy of its first V tile, so every wait for that tile runs
+ * out after the limit set by attn_set_wait_limit_ms; the kernel then records
+ * ATTN_DEVICE_TIMEOUT_BASE + 20 in the status word, leaves no copy in flight
+ * and returns, and attn_sync_status() reports ATTN_ERR_TIMEOUT.  The output
+ * of such a call is undefined.  which = 0 restores normal operation (the
+ * default).  Other values: ATTN_ERR_INVALID_ARG.  Not thread-safe with
+ * respect to calls in flight on other host threads. */
+ATTN_API int attn_test_withhold_copy(int which);
+
 /* Human-readable name of a status code (static string). */
 ATTN_API const char* attn_status_string(int status);
 
