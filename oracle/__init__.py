@@ -65,7 +65,7 @@ def _load(path: str | None = None):
                                    ci, ci, i32p, ctypes.c_int64, f64p, f64p, u8p, f64p, f64p, ci]
     lib.oracle_decode.restype = ci
     lib.oracle_decode.argtypes = [u16p, u16p, u16p, ci, ci, ci, ci, ci, ctypes.c_double, ci, ci,
-                                  f64p, f64p, u8p, f64p, f64p, ci]
+                                  ci, f64p, f64p, u8p, f64p, f64p, ci]
     if path is None:
         _lib = lib
     return lib
@@ -124,12 +124,17 @@ def prefill(Q, K, V, causal: bool, tau: float, Br: int, Bc: int, units=None,
     return out
 
 
+RULE_PER_HEAD = 1   # each query head takes the test on its own row
+RULE_SINK_SEED = 2  # each split's running max starts at the first key tile's max
+
+
 def decode(q, K, V, tau: float, Ls: int, Bt: int = 64, want_exact: bool = True,
-           nthreads: int = 0, lib_path: str | None = None) -> dict:
+           nthreads: int = 0, lib_path: str | None = None, rule: int = 0) -> dict:
     """fp64 Skip Softmax decode.  q [B,Hq,d], K/V [B,Hkv,L,d] (bf16).
 
-    Returns ``o`` [B,Hq,d], ``mask``/``margin`` [B,Hkv,ceil(L/Bt)], and when
-    ``want_exact`` ``o_exact`` and ``pskip`` [B,Hq].
+    Returns ``o`` [B,Hq,d], ``mask``/``margin`` [B,Hkv,ceil(L/Bt)] ([B,Hq,...]
+    with RULE_PER_HEAD), and when ``want_exact`` ``o_exact`` and ``pskip`` [B,Hq].
+    ``rule`` selects the decode rule variant (bits RULE_PER_HEAD, RULE_SINK_SEED).
     """
     qb, k, v = _bits(q), _bits(K), _bits(V)
     B, Hq, d = qb.shape
@@ -138,11 +143,13 @@ def decode(q, K, V, tau: float, Ls: int, Bt: int = 64, want_exact: bool = True,
     o = np.full((B, Hq, d), np.nan)
     o_exact = np.full((B, Hq, d), np.nan) if want_exact else None
     pskip = np.full((B, Hq), np.nan) if want_exact else None
-    mask = np.full((B, Hkv, n_t), 255, dtype=np.uint8)
-    margin = np.full((B, Hkv, n_t), np.nan)
+    rows = Hq if rule & RULE_PER_HEAD else Hkv
+    mask = np.full((B, rows, n_t), 255, dtype=np.uint8)
+    margin = np.full((B, rows, n_t), np.nan)
     lib = _load(lib_path)
     st = lib.oracle_decode(_p(qb, ctypes.c_uint16), _p(k, ctypes.c_uint16), _p(v, ctypes.c_uint16),
-                           B, Hq, Hkv, L, d, float(tau), int(Ls), int(Bt), _p(o, ctypes.c_double),
+                           B, Hq, Hkv, L, d, float(tau), int(Ls), int(Bt), int(rule),
+                           _p(o, ctypes.c_double),
                            _p(o_exact, ctypes.c_double), _p(mask, ctypes.c_uint8),
                            _p(margin, ctypes.c_double), _p(pskip, ctypes.c_double), int(nthreads))
     if st != 0:

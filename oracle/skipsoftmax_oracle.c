@@ -33,6 +33,16 @@
  *     head; the key range is cut into splits of Ls keys, each split runs the
  *     tile loop with its own running max starting at -inf, and the split
  *     results are merged exactly (log-sum-exp).
+ *   - decode rule variants (bits of `rule`; 0 is the rule above):
+ *       ORACLE_RULE_PER_HEAD: each query head takes the test on its own row
+ *         (skips its own exponentials and value sums); the shared value tile
+ *         is needed iff some head of the group keeps the tile.  Mask and
+ *         margin are then per query head, [B, Hq, tiles].
+ *       ORACLE_RULE_SINK_SEED: every split's running max starts at the row
+ *         maximum over the first key tile of the sequence (keys [0, Bt)),
+ *         where attention sinks sit, instead of -inf; a split's first tile
+ *         can then be skipped.  With one split (Ls >= L) this changes
+ *         nothing, as tile 0 is that split's first tile.
  *
  * Every floating-point quantity is fp64; inputs are bf16 bit patterns that are
  * widened exactly.
@@ -48,6 +58,8 @@
 #define ORACLE_OK 0
 #define ORACLE_BAD_ARG 1
 #define ORACLE_NO_MEMORY 2
+#define ORACLE_RULE_PER_HEAD 1
+#define ORACLE_RULE_SINK_SEED 2
 
 /* bf16 -> fp64: a bf16 value is the top half of an IEEE fp32 word. */
 static double widen_bf16(uint16_t bits)
@@ -265,13 +277,17 @@ int oracle_prefill(const uint16_t *Q, const uint16_t *K, const uint16_t *V,
  * heads of one KV head.  Splits of Ls keys, tiles of Bt keys inside a split.
  * o [B,Hq,d] fp64.  Optional: o_exact [B,Hq,d]; mask/margin [B,Hkv,ceil(L/Bt)]
  * (tiles are numbered globally: tile j covers keys [j*Bt, (j+1)*Bt) cut at the
- * split end, so Ls must be a multiple of Bt); pskip [B,Hq].
+ * split end, so Ls must be a multiple of Bt); pskip [B,Hq].  With
+ * ORACLE_RULE_PER_HEAD in `rule`, mask and margin are [B,Hq,ceil(L/Bt)].
  */
 int oracle_decode(const uint16_t *q, const uint16_t *K, const uint16_t *V,
                   int B, int Hq, int Hkv, int L, int d, double tau, int Ls, int Bt,
-                  double *o, double *o_exact, uint8_t *mask, double *margin,
+                  int rule, double *o, double *o_exact, uint8_t *mask, double *margin,
                   double *pskip, int nthreads)
 {
+    const int per_head = (rule & ORACLE_RULE_PER_HEAD) != 0;
+    const int seeded = (rule & ORACLE_RULE_SINK_SEED) != 0;
+    if (rule & ~(ORACLE_RULE_PER_HEAD | ORACLE_RULE_SINK_SEED)) return ORACLE_BAD_ARG;
     if (!q || !K || !V || !o) return ORACLE_BAD_ARG;
     if (B <= 0 || Hq <= 0 || Hkv <= 0 || L <= 0 || d <= 0 || Ls <= 0 || Bt <= 0) return ORACLE_BAD_ARG;
     if (Hq % Hkv != 0 || Ls % Bt != 0) return ORACLE_BAD_ARG;
@@ -298,11 +314,13 @@ int oracle_decode(const uint16_t *q, const uint16_t *K, const uint16_t *V,
         double *sl = malloc(sizeof(double) * (size_t)n_splits * g);   /* per-split sum   */
         double *sa = malloc(sizeof(double) * (size_t)n_splits * g * d);/* per-split acc  */
         double *mt = malloc(sizeof(double) * g);
-        uint8_t *skipped = calloc(n_tiles, 1);
-        if (!s || !m || !l || !acc || !sm || !sl || !sa || !mt || !skipped) {
+        uint8_t *skipped = calloc((size_t)n_tiles * g, 1);  /* [row][tile] */
+        double *seed = malloc(sizeof(double) * g);
+        if (!s || !m || !l || !acc || !sm || !sl || !sa || !mt || !skipped || !seed) {
 #pragma omp critical
             status = ORACLE_NO_MEMORY;
             free(s); free(m); free(l); free(acc); free(sm); free(sl); free(sa); free(mt); free(skipped);
+            free(seed);
             continue;
         }
         for (int c = 0; c < L; ++c)
@@ -310,9 +328,15 @@ int oracle_decode(const uint16_t *q, const uint16_t *K, const uint16_t *V,
                 const uint16_t *qr = q + ((size_t)b * Hq + (size_t)kvh * g + r) * d;
                 s[(size_t)c * g + r] = dot_widened(qr, k + (size_t)c * d, d) * inv_sqrt_d;
             }
+        /* sink seed: row maximum over the first key tile of the sequence */
+        for (int r = 0; r < g; ++r) {
+            seed[r] = -INFINITY;
+            for (int c = 0; c < Bt && c < L; ++c)
+                if (s[(size_t)c * g + r] > seed[r]) seed[r] = s[(size_t)c * g + r];
+        }
         for (int sp = 0; sp < n_splits; ++sp) {
             const int k0 = sp * Ls, k1 = (k0 + Ls < L) ? k0 + Ls : L;
-            for (int r = 0; r < g; ++r) { m[r] = -INFINITY; l[r] = 0.0; }
+            for (int r = 0; r < g; ++r) { m[r] = seeded ? seed[r] : -INFINITY; l[r] = 0.0; }
             for (size_t t = 0; t < (size_t)g * d; ++t) acc[t] = 0.0;
             for (int c0 = k0; c0 < k1; c0 += Bt) {
                 const int c1 = (c0 + Bt < k1) ? c0 + Bt : k1;
@@ -325,12 +349,29 @@ int oracle_decode(const uint16_t *q, const uint16_t *K, const uint16_t *V,
                     double x = row_margin(mt[r], m[r], tau);
                     if (x > margin_j) margin_j = x;
                 }
-                const int skip = margin_j < 0.0;
-                const size_t ti = (size_t)(b * Hkv + kvh) * n_tiles + j;
-                if (mask) mask[ti] = (uint8_t)skip;
-                if (margin) margin[ti] = margin_j;
-                if (skip) { skipped[j] = 1; continue; }
+                if (per_head) {
+                    /* each row decides for itself; margins per query head */
+                    for (int r = 0; r < g; ++r) {
+                        const double x = row_margin(mt[r], m[r], tau);
+                        const size_t ti = ((size_t)b * Hq + (size_t)kvh * g + r) * n_tiles + j;
+                        if (mask) mask[ti] = (uint8_t)(x < 0.0);
+                        if (margin) margin[ti] = x;
+                    }
+                } else {
+                    const int skip = margin_j < 0.0;
+                    const size_t ti = (size_t)(b * Hkv + kvh) * n_tiles + j;
+                    if (mask) mask[ti] = (uint8_t)skip;
+                    if (margin) margin[ti] = margin_j;
+                    if (skip) {
+                        for (int r = 0; r < g; ++r) skipped[(size_t)r * n_tiles + j] = 1;
+                        continue;
+                    }
+                }
                 for (int r = 0; r < g; ++r) {
+                    if (per_head && row_margin(mt[r], m[r], tau) < 0.0) {
+                        skipped[(size_t)r * n_tiles + j] = 1;
+                        continue;
+                    }
                     const double m_new = (mt[r] > m[r]) ? mt[r] : m[r];
                     const double alpha = (m[r] == -INFINITY) ? 0.0 : exp(m[r] - m_new);
                     l[r] *= alpha;
@@ -358,6 +399,7 @@ int oracle_decode(const uint16_t *q, const uint16_t *K, const uint16_t *V,
             double *orow = o + ((size_t)b * Hq + (size_t)kvh * g + r) * d;
             for (int t = 0; t < d; ++t) orow[t] = 0.0;
             for (int sp = 0; sp < n_splits; ++sp) {
+                if (sl[(size_t)sp * g + r] == 0.0) continue;  /* every tile of the split skipped */
                 const double w = exp(sm[(size_t)sp * g + r] - M);
                 den += w * sl[(size_t)sp * g + r];
                 for (int t = 0; t < d; ++t) orow[t] += w * sa[((size_t)sp * g + r) * d + t];
@@ -374,7 +416,7 @@ int oracle_decode(const uint16_t *q, const uint16_t *K, const uint16_t *V,
                 for (int c = 0; c < L; ++c) {
                     const double p = exp(s[(size_t)c * g + r] - M);
                     total += p;
-                    if (skipped[c / Bt]) lost += p;
+                    if (skipped[(size_t)r * n_tiles + c / Bt]) lost += p;
                     for (int t = 0; t < d; ++t) acc[t] += p * widen_bf16(v[(size_t)c * d + t]);
                 }
                 const size_t row = (size_t)b * Hq + (size_t)kvh * g + r;
@@ -383,6 +425,7 @@ int oracle_decode(const uint16_t *q, const uint16_t *K, const uint16_t *V,
             }
         }
         free(s); free(m); free(l); free(acc); free(sm); free(sl); free(sa); free(mt); free(skipped);
+        free(seed);
     }
     return status;
 }

@@ -24,9 +24,14 @@ MUTANTS = {
     "causal_off_by_one": ("if (a->causal && c > qi) x = -INFINITY;", "if (a->causal && c >= qi && qi > 0) x = -INFINITY;"),
     "transposed_value_rows": ("ar[t] += p * widen_bf16(vc[t]);", "ar[t] += p * widen_bf16(v[(size_t)t * d + (c % d)]);"),
     "decode_max_not_reset_per_split": (
-        "for (int r = 0; r < g; ++r) { m[r] = -INFINITY; l[r] = 0.0; }\n            for (size_t t",
-        "for (int r = 0; r < g; ++r) { if (sp == 0) m[r] = -INFINITY; l[r] = 0.0; }\n            for (size_t t"),
+        "for (int r = 0; r < g; ++r) { m[r] = seeded ? seed[r] : -INFINITY; l[r] = 0.0; }\n            for (size_t t",
+        "for (int r = 0; r < g; ++r) { if (sp == 0) m[r] = seeded ? seed[r] : -INFINITY; l[r] = 0.0; }\n            for (size_t t"),
     "decode_merge_unweighted_sum": ("den += w * sl[(size_t)sp * g + r];", "den += sl[(size_t)sp * g + r];"),
+    "per_head_uses_group_margin": (
+        "if (per_head && row_margin(mt[r], m[r], tau) < 0.0) {",
+        "if (per_head && margin_j < 0.0) {"),
+    "sink_seed_from_second_tile": (
+        "for (int c = 0; c < Bt && c < L; ++c)", "for (int c = Bt; c < 2 * Bt && c < L; ++c)"),
 }
 
 

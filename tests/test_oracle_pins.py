@@ -406,6 +406,80 @@ def pin_decode_matches_prefill_single_row(lib):
         np.testing.assert_array_equal(d_["mask"][0, 0], p_["mask"][0, 0, 0])
 
 
+def dec_brute(s, V, g, Ls, Bt, tau, per_head, seeded):
+    """Decode decisions and output from the definition of each rule variant.
+
+    Per head: row r of a KV group skips tile j iff its running max m_r (the
+    max over the split's earlier tiles, and with seeding also over keys
+    [0, Bt)) exists and the tile max is below m_r - tau.  Group rule: the tile
+    is skipped iff every row of the group would skip it.  Returns the mask
+    ([B,Hq,T] per head, [B,Hkv,T] group) and softmax over each row's kept keys."""
+    B, Hq, L = s.shape
+    T = -(-L // Bt)
+    mask = np.zeros((B, Hq if per_head else Hq // g, T), np.uint8)
+    keep = np.zeros_like(s, bool)
+    for b in range(B):
+        for kv in range(Hq // g):
+            rows = s[b, kv * g:(kv + 1) * g]
+            seed = rows[:, :min(Bt, L)].max(-1)
+            for j in range(T):
+                c0, c1 = j * Bt, min(L, j * Bt + Bt)
+                split0 = (c0 // Ls) * Ls
+                m = rows[:, split0:c0].max(-1) if c0 > split0 else np.full(g, -np.inf)
+                if seeded:
+                    m = np.maximum(m, seed)
+                mt = rows[:, c0:c1].max(-1)
+                row_skip = np.array([mm != -np.inf and t < mm - tau for t, mm in zip(mt, m)])
+                if per_head:
+                    mask[b, kv * g:(kv + 1) * g, j] = row_skip
+                    for r in range(g):
+                        keep[b, kv * g + r, c0:c1] = not row_skip[r]
+                else:
+                    mask[b, kv, j] = row_skip.all()
+                    keep[b, kv * g:(kv + 1) * g, c0:c1] = not row_skip.all()
+    w = np.where(keep, np.exp(s - s.max(-1, keepdims=True)), 0.0)
+    v = np.repeat(f64(V), g, axis=1)
+    return mask, np.einsum("bhk,bhkd->bhd", w, v) / w.sum(-1, keepdims=True)
+
+
+@pin
+def pin_decode_rule_variants_from_definition(lib):
+    """Per-head and sink-seeded decode rules equal their definitions; the
+    error bound holds per row; per-head skips a superset (per row) of the
+    group rule, seeding a superset of the unseeded rule; per-head with g = 1
+    and seeding with a single split change nothing."""
+    q, K, V = dec_inputs(L=700)
+    s = dec_scores(q, K)
+    g, Bt = 2, 64
+    vmax = np.abs(f64(V)).max()
+    saw = {1: False, 2: False, 3: False}
+    for Ls in (128, 320, 704):
+        for tau in (0.0, 2.0, 6.0):
+            base = oracle.decode(q, K, V, tau, Ls, Bt, lib_path=lib)
+            for rule in (1, 2, 3):
+                r = oracle.decode(q, K, V, tau, Ls, Bt, lib_path=lib, rule=rule)
+                mask, ref = dec_brute(s, V, g, Ls, Bt, tau, rule & 1, rule & 2)
+                np.testing.assert_array_equal(r["mask"], mask)
+                np.testing.assert_allclose(r["o"], ref, rtol=0, atol=1e-12)
+                dev = np.abs(r["o"] - r["o_exact"]).max(-1)
+                assert np.all(dev <= 2 * vmax * r["pskip"] + 1e-12)
+                saw[rule] |= bool((r["mask"] == 1).any())
+                gm = np.repeat(base["mask"], g, axis=1) if rule & 1 else base["mask"]
+                if rule in (1, 2):  # a superset of the base rule's skips
+                    assert np.all(r["mask"][gm == 1] == 1)
+            if Ls >= 700:  # one split: seeding changes nothing
+                seeded = oracle.decode(q, K, V, tau, Ls, Bt, lib_path=lib, rule=2)
+                np.testing.assert_array_equal(seeded["mask"], base["mask"])
+                np.testing.assert_allclose(seeded["o"], base["o"], rtol=0, atol=1e-13)
+    assert all(saw.values())
+    q1, K1, V1 = dec_inputs(Hq=2, Hkv=2, L=500, seed=21)  # g = 1: per head is the group rule
+    for tau in (1.0, 4.0):
+        a = oracle.decode(q1, K1, V1, tau, 192, Bt, lib_path=lib)
+        b_ = oracle.decode(q1, K1, V1, tau, 192, Bt, lib_path=lib, rule=1)
+        np.testing.assert_array_equal(a["mask"], b_["mask"])
+        np.testing.assert_allclose(a["o"], b_["o"], rtol=0, atol=1e-13)
+
+
 @pytest.mark.parametrize("fn", PINS, ids=[f.__name__ for f in PINS])
 def test_pin(fn):
     fn(None)
