@@ -19,7 +19,7 @@ import os
 
 __all__ = [
     "AttnError", "lib", "attn_prefill", "attn_prefill_ex", "attn_decode", "attn_decode_ex",
-    "attn_decode_noalloc",
+    "attn_decode_noalloc", "attn_decode_rule", "RULE_GROUP", "RULE_PER_HEAD", "RULE_SINK_SEED",
     "attn_decode_split_len", "attn_decode_tile", "attn_decode_workspace_bytes",
     "attn_set_stream", "attn_sync_status", "attn_last_timeout_site", "attn_set_wait_limit_ms",
     "attn_test_withhold_copy", "attn_status_string", "attn_shutdown", "prefill", "decode", "STATUS",
@@ -55,6 +55,7 @@ def lib() -> ctypes.CDLL:
         "attn_decode": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf]),
         "attn_decode_ex": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, vp, vp, vp, sz]),
         "attn_decode_noalloc": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, vp, vp]),
+        "attn_decode_rule": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, vp, vp, vp, sz]),
         "attn_decode_split_len": (ci, [ci, ci, ci]),
         "attn_decode_tile": (ci, []),
         "attn_decode_workspace_bytes": (sz, [ci, ci, ci, ci, ci]),
@@ -90,6 +91,15 @@ def attn_decode(q, K, V, o, B, Hq, Hkv, L, d, tau) -> int:
 
 def attn_decode_ex(q, K, V, o, B, Hq, Hkv, L, d, tau, stream=None, skip_mask=None, ws=None, ws_bytes=0) -> int:
     return lib().attn_decode_ex(q, K, V, o, B, Hq, Hkv, L, d, float(tau), stream, skip_mask, ws, ws_bytes)
+
+
+RULE_GROUP, RULE_PER_HEAD, RULE_SINK_SEED = 0, 1, 2
+
+
+def attn_decode_rule(q, K, V, o, B, Hq, Hkv, L, d, tau, rule, stream=None, skip_mask=None, ws=None,
+                     ws_bytes=0) -> int:
+    return lib().attn_decode_rule(q, K, V, o, B, Hq, Hkv, L, d, float(tau), int(rule), stream,
+                                  skip_mask, ws, ws_bytes)
 
 
 def attn_decode_noalloc(q, K, V, o, B, Hq, Hkv, L, d, tau, stream=None, skip_mask=None) -> int:
@@ -177,7 +187,7 @@ def prefill(Q, K, V, causal: bool, tau: float = math.inf, Br: int = 128, Bc: int
 
 
 def decode(q, K, V, tau: float = math.inf, out=None, skip_mask: bool = False, stream=None,
-           workspace=None):
+           workspace=None, rule: int = RULE_GROUP):
     """o = Skip Softmax decode attention: q [B,Hq,d], K/V [B,Hkv,L,d] bf16 CUDA tensors.
 
     ``workspace``: optional uint8 CUDA tensor of at least
@@ -193,10 +203,11 @@ def decode(q, K, V, tau: float = math.inf, out=None, skip_mask: bool = False, st
     o = out if out is not None else torch.empty_like(q)
     mask = None
     if skip_mask:
-        mask = torch.empty(B, Hkv, -(-L // attn_decode_tile()), dtype=torch.uint8, device=q.device)
+        rows = Hq if rule & RULE_PER_HEAD else Hkv
+        mask = torch.empty(B, rows, -(-L // attn_decode_tile()), dtype=torch.uint8, device=q.device)
     ws, wsb = (None, 0) if workspace is None else (workspace.data_ptr(), workspace.numel())
-    st = attn_decode_ex(q.data_ptr(), K.data_ptr(), V.data_ptr(), o.data_ptr(), B, Hq, Hkv, L, d,
-                        tau, _stream_ptr(stream), mask.data_ptr() if mask is not None else None,
-                        ws, wsb)
-    _check(st, "attn_decode_ex")
+    st = attn_decode_rule(q.data_ptr(), K.data_ptr(), V.data_ptr(), o.data_ptr(), B, Hq, Hkv, L, d,
+                          tau, rule, _stream_ptr(stream),
+                          mask.data_ptr() if mask is not None else None, ws, wsb)
+    _check(st, "attn_decode_rule")
     return (o, mask) if skip_mask else o

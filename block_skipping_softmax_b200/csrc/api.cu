@@ -178,6 +178,14 @@ size_t attn_decode_workspace_bytes(int B, int Hq, int Hkv, int L, int d) {
 int attn_decode_ex(const void* q, const void* K, const void* V, void* o, int B, int Hq, int Hkv,
                    int L, int d, float tau, void* stream, uint8_t* skip_mask, void* ws,
                    size_t ws_bytes) {
+  return attn_decode_rule(q, K, V, o, B, Hq, Hkv, L, d, tau, ATTN_DECODE_RULE_GROUP, stream,
+                          skip_mask, ws, ws_bytes);
+}
+
+int attn_decode_rule(const void* q, const void* K, const void* V, void* o, int B, int Hq, int Hkv,
+                     int L, int d, float tau, int rule, void* stream, uint8_t* skip_mask, void* ws,
+                     size_t ws_bytes) {
+  if (rule & ~(ATTN_DECODE_RULE_PER_HEAD | ATTN_DECODE_RULE_SINK_SEED)) return ATTN_ERR_INVALID_ARG;
   int st = check_decode(q, K, V, o, B, Hq, Hkv, L, d, tau);
   if (st != ATTN_OK) return st;
   if (ws == nullptr && ws_bytes != 0) return ATTN_ERR_INVALID_ARG;
@@ -227,6 +235,7 @@ int attn_decode_ex(const void* q, const void* K, const void* V, void* o, int B, 
   a.status = status;
   a.wait_limit_ns = g_wait_limit_ns;
   a.stream = static_cast<cudaStream_t>(stream);
+  a.rule = rule;
   {
     std::lock_guard<std::mutex> lk(g_mu);
     a.withhold_v = g_withhold_v;

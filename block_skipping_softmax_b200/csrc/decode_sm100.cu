@@ -87,7 +87,7 @@ struct DecCfg {
   static constexpr int kOffL = kOffW + 2 * kWarps * G * 4;             // float [warps][G]
   static constexpr int kOffMisc = kOffL + kWarps * G * 4;
   static constexpr int kOffBar = kOffMisc + 16;
-  static constexpr int kSmemUsed = kOffBar + 8 * (kKStages + kVStages);
+  static constexpr int kSmemUsed = kOffBar + 8 * (kKStages + kVStages + 1);  // + sink-seed tile
   static constexpr int kSmemBytes = kSmemUsed + 1024;  // room to align the base
   static_assert(G <= kP, "a lane ends the butterfly with one row");
   static_assert(kSIters >= 1 && kKPI * kSIters == kKeysPerWarp, "score lane layout");
@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
                           float* __restrict__ lse_part, uint8_t* __restrict__ skip_mask,
                           int* __restrict__ status, int Hq, int Hkv, int L, int split_len,
                           int n_splits, float scale_log2, float tau_log2, int tau_is_inf,
-                          unsigned long long wait_limit_ns, int withhold_v) {
+                          unsigned long long wait_limit_ns, int withhold_v, int rule) {
   using C = DecCfg<D, G>;
   constexpr unsigned FULL = 0xffffffffu;
   constexpr int kLog2P = ilog2(C::kP);
@@ -158,6 +158,8 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
   const uint32_t bar0 = sbase + C::kOffBar;
   auto b_k_full = [&](int s) { return bar0 + 8u * s; };
   auto b_v_full = [&](int s) { return bar0 + 8u * (kKStages + s); };
+  const uint32_t b_seed = bar0 + 8u * (kKStages + kVStages);
+  const bool per_head = (rule & ATTN_DECODE_RULE_PER_HEAD) != 0;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -183,6 +185,7 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
   if (tid == 0) {
     for (int s = 0; s < kKStages; ++s) mbar_init(b_k_full(s), 1);
     for (int s = 0; s < kVStages; ++s) mbar_init(b_v_full(s), 1);
+    mbar_init(b_seed, 1);
     *never = 0;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -237,6 +240,88 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
   int pv_count = 0;        // V tiles consumed
   bool ok = true;          // this thread's waits so far succeeded
 
+  // Scores of one K tile in shared memory (keys >= key_lim are past L and
+  // read as -inf) into sv; returns this warp's maximum for row_q.
+  auto tile_scores = [&](const uint8_t* kt, int key_lim, float (&sv)[C::kSIters]) -> float {
+    float wm = NEG_INF;
+#pragma unroll
+    for (int it = 0; it < C::kSIters; ++it) {
+      const int key = warp * C::kKeysPerWarp + it * C::kKPI + kl;
+      float2 s2[G];
+#pragma unroll
+      for (int r = 0; r < G; ++r) s2[r] = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < C::kCPL; ++j) {
+        const uint4 u = *reinterpret_cast<const uint4*>(kt + chunk_off<D>(key, j * C::kP + qd));
+        float2 kf[4];
+        bf16x8_to_f32(u, kf);
+#pragma unroll
+        for (int r = 0; r < G; ++r)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) s2[r] = __ffma2_rn(qf[r][j][e], kf[e], s2[r]);
+      }
+      float v[G];
+#pragma unroll
+      for (int r = 0; r < G; ++r) v[r] = s2[r].x + s2[r].y;
+      // butterfly over the kP lanes of this key, highest qd bit first: the
+      // first log2(G) steps each keep half of the rows (the lanes with the
+      // bit set keep the upper half), the rest are plain sums
+#pragma unroll
+      for (int s = 0; s < kLog2P; ++s) {
+        const int qbit = kLog2P - 1 - s;
+        const int o = C::kKeyMajor ? (1 << qbit) : (C::kKPI << qbit);
+        const int n = G >> s;
+        if (n > 1) {
+          const int hh = n / 2;
+          const bool upper = ((qd >> qbit) & 1) != 0;
+#pragma unroll
+          for (int r = 0; r < hh; ++r) {
+            const float send = upper ? v[r] : v[r + hh];
+            const float keep = upper ? v[r + hh] : v[r];
+            v[r] = keep + __shfl_xor_sync(FULL, send, o);
+          }
+        } else {
+          v[0] += __shfl_xor_sync(FULL, v[0], o);
+        }
+      }
+      sv[it] = key < key_lim ? v[0] : NEG_INF;
+      wm = fmaxf(wm, sv[it]);
+    }
+    // max over the warp's keys for row_q
+    if constexpr (C::kKeyMajor) {
+#pragma unroll
+      for (int o = C::kP; o < 32; o <<= 1) wm = fmaxf(wm, __shfl_xor_sync(FULL, wm, o));
+    } else {
+#pragma unroll
+      for (int o = 1; o < C::kKPI; o <<= 1) wm = fmaxf(wm, __shfl_xor_sync(FULL, wm, o));
+    }
+    return wm;
+  };
+
+  // Sink seed: the running max of a split other than the first starts at the
+  // rows' maximum over the sequence's first key tile (where attention sinks
+  // sit) instead of -inf.  The tile goes to V slot 0, free until the first
+  // V copy, which is issued only after the first decision.
+  bool seed_issued = false;
+  if ((rule & ATTN_DECODE_RULE_SINK_SEED) && t_begin > 0) {
+    if (tid == 0) {
+      issue(sbase + C::kOffV, &tmK, b_seed, 0);
+      seed_issued = true;
+    }
+    const bool got = mbar_wait(b_seed, 0, never, wait_limit_ns);
+    ok = ok && got;
+    float sv0[C::kSIters];
+    const float wm0 = tile_scores(smem + C::kOffV, L, sv0);
+    if (kl == 0 && leader) wmax[(kWarps + warp) * G + row_q] = wm0;  // buffer 1; tile 0 uses buffer 0
+    __syncthreads();
+    const float* wb = wmax + kWarps * G;
+    float mt = lane < n_dec ? wb[lane] : NEG_INF;
+    if constexpr (G == 8) mt = fmaxf(mt, wb[lane + 32]);
+#pragma unroll
+    for (int o = G; o < n_dec; o <<= 1) mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, o));
+    m_exact = lane < n_dec ? mt : NEG_INF;
+  }
+
   for (int i = 0; i < nt + kLag; ++i) {
     // ---------------- A: scores of tile i and the per-warp row maxima
     float sv[C::kSIters];
@@ -246,58 +331,7 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
       ok = ok && got;  // on a give-up the scores are garbage and dropped at the barrier
       const uint8_t* kt = smem + C::kOffK + ks * C::kTileBytes;
       const int key_lim = L - (t_begin + i) * kDecodeTile;  // keys >= key_lim are past L
-      float wm = NEG_INF;
-#pragma unroll
-      for (int it = 0; it < C::kSIters; ++it) {
-        const int key = warp * C::kKeysPerWarp + it * C::kKPI + kl;
-        float2 s2[G];
-#pragma unroll
-        for (int r = 0; r < G; ++r) s2[r] = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int j = 0; j < C::kCPL; ++j) {
-          const uint4 u = *reinterpret_cast<const uint4*>(kt + chunk_off<D>(key, j * C::kP + qd));
-          float2 kf[4];
-          bf16x8_to_f32(u, kf);
-#pragma unroll
-          for (int r = 0; r < G; ++r)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) s2[r] = __ffma2_rn(qf[r][j][e], kf[e], s2[r]);
-        }
-        float v[G];
-#pragma unroll
-        for (int r = 0; r < G; ++r) v[r] = s2[r].x + s2[r].y;
-        // butterfly over the kP lanes of this key, highest qd bit first: the
-        // first log2(G) steps each keep half of the rows (the lanes with the
-        // bit set keep the upper half), the rest are plain sums
-#pragma unroll
-        for (int s = 0; s < kLog2P; ++s) {
-          const int qbit = kLog2P - 1 - s;
-          const int o = C::kKeyMajor ? (1 << qbit) : (C::kKPI << qbit);
-          const int n = G >> s;
-          if (n > 1) {
-            const int hh = n / 2;
-            const bool upper = ((qd >> qbit) & 1) != 0;
-#pragma unroll
-            for (int r = 0; r < hh; ++r) {
-              const float send = upper ? v[r] : v[r + hh];
-              const float keep = upper ? v[r + hh] : v[r];
-              v[r] = keep + __shfl_xor_sync(FULL, send, o);
-            }
-          } else {
-            v[0] += __shfl_xor_sync(FULL, v[0], o);
-          }
-        }
-        sv[it] = key < key_lim ? v[0] : NEG_INF;
-        wm = fmaxf(wm, sv[it]);
-      }
-      // max over the warp's keys for row_q
-      if constexpr (C::kKeyMajor) {
-#pragma unroll
-        for (int o = C::kP; o < 32; o <<= 1) wm = fmaxf(wm, __shfl_xor_sync(FULL, wm, o));
-      } else {
-#pragma unroll
-        for (int o = 1; o < C::kKPI; o <<= 1) wm = fmaxf(wm, __shfl_xor_sync(FULL, wm, o));
-      }
+      const float wm = tile_scores(kt, key_lim, sv);
       if (kl == 0 && leader) wmax[((i & 1) * kWarps + warp) * G + row_q] = wm;
     }
     if (__syncthreads_or(!ok)) {  // the single per-tile barrier; also a uniform give-up
@@ -316,6 +350,8 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
       const bool pass =
           lane >= n_dec || (m_exact != NEG_INF && (mt == NEG_INF || mt < m_exact - tau_log2));
       keep_i = tau_is_inf || !__all_sync(FULL, pass);
+      // per-head rule: bit r set iff row r computes this tile (lanes 0..G-1 hold rows 0..G-1)
+      const unsigned row_keep = (per_head && !tau_is_inf) ? __ballot_sync(FULL, !pass) : 0xffffffffu;
       m_exact = fmaxf(m_exact, mt);  // a skipped tile never raises it
       if (keep_i) {
         const bool moved = m_exact > m_ref + kRefSlack;
@@ -335,16 +371,19 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
 #pragma unroll
         for (int it = 0; it < C::kSIters; ++it) {
           const int key = warp * C::kKeysPerWarp + it * C::kKPI + kl;
-          const float p = ex2(sv[it] - mr);
+          const float p = ((row_keep >> row_q) & 1u) ? ex2(sv[it] - mr) : 0.f;
           if (leader) {
             pr[key * G + row_q] = p;
             lsum += p;
           }
         }
       }
+      if (per_head && skip_mask && warp == 0 && lane < G)  // one mask entry per query head
+        skip_mask[(static_cast<size_t>(b) * Hq + kv * G + lane) * n_tiles_all + t_begin + i] =
+            (keep_i && ((row_keep >> lane) & 1u)) ? 0 : 1;
       if (tid == 0) {
         const int t = t_begin + i;
-        if (skip_mask) skip_mask[static_cast<size_t>(bh) * n_tiles_all + t] = keep_i ? 0 : 1;
+        if (skip_mask && !per_head) skip_mask[static_cast<size_t>(bh) * n_tiles_all + t] = keep_i ? 0 : 1;
         if (keep_i) {  // the slot's previous tile finished its P*V before this barrier
           const int vs = v_issued % kVStages;
           // test support: the first copy can be withheld, so that every wait
@@ -417,6 +456,7 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
       for (int k = max(0, v_issued - kVStages); k < v_issued; ++k)
         if (!(withhold_v && k == 0))  // a withheld copy was never issued
           mbar_drain(b_v_full(k % kVStages), (k / kVStages) & 1, wait_limit_ns);
+      if (seed_issued) mbar_drain(b_seed, 0, wait_limit_ns);
     }
     return;
   }
@@ -465,7 +505,9 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
       den += wl[w * G + r];
     }
     const size_t row = static_cast<size_t>(b) * Hq + kv * G + r;
-    o_part[(row * n_splits + split) * D + col] = s / den;
+    // a row that skipped every tile of its split (possible with the sink seed
+    // or the per-head rule) contributes nothing to the merge
+    o_part[(row * n_splits + split) * D + col] = den > 0.f ? s / den : 0.f;
   }
   if (tid < G) {
     // lane tid of warp 0 holds the reference max of row tid, which is the one
@@ -474,7 +516,7 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) den += wl[w * G + tid];
     const size_t row = static_cast<size_t>(b) * Hq + kv * G + tid;
-    lse_part[row * n_splits + split] = m_ref + __log2f(den);
+    lse_part[row * n_splits + split] = den > 0.f ? m_ref + __log2f(den) : NEG_INF;
   }
 }
 
@@ -548,7 +590,7 @@ int launch_dg(const DecodeLaunch& a) {
   kern<<<grid, kDecThreads, C::kSmemBytes, a.stream>>>(
       mk, mv, static_cast<const __nv_bfloat16*>(a.q), a.o_part, a.lse_part, a.skip_mask,
       a.status, a.Hq, a.Hkv, a.L, a.split_len, a.n_splits, a.scale_log2, a.tau_log2,
-      a.tau_is_inf, a.wait_limit_ns, a.withhold_v);
+      a.tau_is_inf, a.wait_limit_ns, a.withhold_v, a.rule);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   decode_combine_kernel<D><<<a.B * a.Hq, D, 0, a.stream>>>(
       a.o_part, a.lse_part, static_cast<__nv_bfloat16*>(a.o), a.n_splits);

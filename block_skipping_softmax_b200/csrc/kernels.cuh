@@ -48,6 +48,7 @@ struct DecodeLaunch {
   unsigned long long wait_limit_ns;
   cudaStream_t stream;
   int withhold_v;  // test support: 1 = every CTA withholds its first V copy
+  int rule;        // ATTN_DECODE_RULE_* bits
 };
 
 int launch_decode(const DecodeLaunch& a);

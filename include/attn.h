@@ -107,6 +107,33 @@ ATTN_API int attn_decode_ex(const void* q, const void* K, const void* V, void* o
                    size_t ws_bytes);
 
 /*
+ * Decode rule variants (bits of `rule` in attn_decode_rule).  The Skip
+ * Softmax page compares a block's local maximum with the running maximum of
+ * each row and says nothing on which rows of a decode step must agree, or
+ * where a split of the key range starts its running maximum:
+ *   ATTN_DECODE_RULE_GROUP (0): the rule of attn_decode above.
+ *   ATTN_DECODE_RULE_PER_HEAD: every query head takes the test on its own row
+ *     and skips its own exponentials and value sums; the V tile is still
+ *     loaded iff some head of the group keeps the tile.  skip_mask is then
+ *     [B, Hq, ceil(L/64)] (1 = that head skipped the tile).
+ *   ATTN_DECODE_RULE_SINK_SEED: the running maximum of every split but the
+ *     first starts at each row's maximum over keys [0, 64) of the sequence
+ *     (where attention sinks sit) instead of -inf, so a split's first tiles
+ *     can be skipped too.  With a single split this changes nothing.
+ */
+#define ATTN_DECODE_RULE_GROUP 0
+#define ATTN_DECODE_RULE_PER_HEAD 1
+#define ATTN_DECODE_RULE_SINK_SEED 2
+
+/*
+ * attn_decode_ex with a rule variant (a combination of the bits above; other
+ * bits: ATTN_ERR_INVALID_ARG).  rule = 0 is exactly attn_decode_ex.
+ */
+ATTN_API int attn_decode_rule(const void* q, const void* K, const void* V, void* o, int B, int Hq,
+                              int Hkv, int L, int d, float tau, int rule, void* stream,
+                              uint8_t* skip_mask, void* ws, size_t ws_bytes);
+
+/*
  * Decode that allocates nothing, for callers that cannot allocate device
  * memory (a serving engine that has reserved all of HBM for its own pools, a
  * latency-critical loop that must not meet the implicit synchronisation of
