@@ -421,6 +421,35 @@ def main():
                          "kernel": "decode_partial_kernel<128,4> + decode_combine_kernel<128>",
                          "algorithmic": "K bytes + kept fraction x V bytes per launch"},
             "split_len": bss.attn_decode_split_len(wd["B"], wd["Hkv"], wd["L"])}
+    # the decode rule variants (per-head test, sink-seeded splits) at the
+    # thresholds where the skip rule acts
+    if not args.quick:
+        g = wd["Hq"] // wd["Hkv"]
+        ls = bss.attn_decode_split_len(wd["B"], wd["Hkv"], wd["L"])
+        n_splits = -(-wd["L"] // ls)
+        variants = {}
+        for rule, rname in ((bss.RULE_PER_HEAD, "per_head"), (bss.RULE_SINK_SEED, "sink_seed"),
+                            (bss.RULE_PER_HEAD | bss.RULE_SINK_SEED, "per_head+sink_seed")):
+            for tau in (2.0, 4.0):
+                ms_v, _, _ = timed(lambda: bss.decode(q, Kd, Vd, tau, out=o, rule=rule),
+                                   max(3, args.steps // 4), 2, f"decode {rname}@tau={tau}")
+                _, mask = bss.decode(q, Kd, Vd, tau, out=o, skip_mask=True, rule=rule)
+                if rule & bss.RULE_PER_HEAD:
+                    m4 = mask.view(wd["B"], wd["Hkv"], g, -1)
+                    v_kept = float((m4 == 0).any(dim=2).float().mean().item())
+                    row_skip = float((mask == 1).float().mean().item())
+                else:
+                    v_kept = 1.0 - float((mask == 1).float().mean().item())
+                    row_skip = 1.0 - v_kept
+                seed_bytes = (wd["B"] * wd["Hkv"] * (n_splits - 1) * 64 * wd["d"] * 2
+                              if rule & bss.RULE_SINK_SEED else 0)
+                read = kv_bytes * (1.0 + v_kept) + seed_bytes
+                gbs = read / (ms_v * 1e-3) / 1e9
+                variants[f"{rname}@tau={tau}"] = {
+                    "value": world * gbs, "unit": "GB/s", "latency_us": ms_v * 1000,
+                    "v_tiles_skipped": 1.0 - v_kept, "row_tiles_skipped": row_skip,
+                    "frac_of_hbm": gbs / peaks["hbm_gbs"]}
+        decode["rule_variants"] = variants
     del q, Kd, Vd, o
     torch.cuda.empty_cache()
 
