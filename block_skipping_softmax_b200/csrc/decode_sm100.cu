@@ -131,7 +131,7 @@ __device__ __forceinline__ void load_row_floats(const float* p, float (&v)[G]) {
 
 }  // namespace
 
-template <int D, int G>
+template <int D, int G, int RULE>
 __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
     decode_partial_kernel(const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV,
@@ -139,7 +139,7 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
                           float* __restrict__ lse_part, uint8_t* __restrict__ skip_mask,
                           int* __restrict__ status, int Hq, int Hkv, int L, int split_len,
                           int n_splits, float scale_log2, float tau_log2, int tau_is_inf,
-                          unsigned long long wait_limit_ns, int withhold_v, int rule) {
+                          unsigned long long wait_limit_ns, int withhold_v) {
   using C = DecCfg<D, G>;
   constexpr unsigned FULL = 0xffffffffu;
   constexpr int kLog2P = ilog2(C::kP);
@@ -159,7 +159,9 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
   auto b_k_full = [&](int s) { return bar0 + 8u * s; };
   auto b_v_full = [&](int s) { return bar0 + 8u * (kKStages + s); };
   const uint32_t b_seed = bar0 + 8u * (kKStages + kVStages);
-  const bool per_head = (rule & ATTN_DECODE_RULE_PER_HEAD) != 0;
+  // the rule variant is a template argument, so the default rule carries no trace of the others
+  constexpr bool per_head = (RULE & ATTN_DECODE_RULE_PER_HEAD) != 0;
+  constexpr bool seeded = (RULE & ATTN_DECODE_RULE_SINK_SEED) != 0;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5;
@@ -303,7 +305,7 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
   // sit) instead of -inf.  The tile goes to V slot 0, free until the first
   // V copy, which is issued only after the first decision.
   bool seed_issued = false;
-  if ((rule & ATTN_DECODE_RULE_SINK_SEED) && t_begin > 0) {
+  if (seeded && t_begin > 0) {
     if (tid == 0) {
       issue(sbase + C::kOffV, &tmK, b_seed, 0);
       seed_issued = true;
@@ -351,7 +353,8 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
           lane >= n_dec || (m_exact != NEG_INF && (mt == NEG_INF || mt < m_exact - tau_log2));
       keep_i = tau_is_inf || !__all_sync(FULL, pass);
       // per-head rule: bit r set iff row r computes this tile (lanes 0..G-1 hold rows 0..G-1)
-      const unsigned row_keep = (per_head && !tau_is_inf) ? __ballot_sync(FULL, !pass) : 0xffffffffu;
+      unsigned row_keep = 0xffffffffu;
+      if constexpr (per_head) row_keep = tau_is_inf ? 0xffffffffu : __ballot_sync(FULL, !pass);
       m_exact = fmaxf(m_exact, mt);  // a skipped tile never raises it
       if (keep_i) {
         const bool moved = m_exact > m_ref + kRefSlack;
@@ -371,7 +374,8 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
 #pragma unroll
         for (int it = 0; it < C::kSIters; ++it) {
           const int key = warp * C::kKeysPerWarp + it * C::kKPI + kl;
-          const float p = ((row_keep >> row_q) & 1u) ? ex2(sv[it] - mr) : 0.f;
+          float p = ex2(sv[it] - mr);
+          if constexpr (per_head) p = ((row_keep >> row_q) & 1u) ? p : 0.f;
           if (leader) {
             pr[key * G + row_q] = p;
             lsum += p;
@@ -570,10 +574,10 @@ bool dec_map(CUtensorMap* m, const void* base, int BH, int L, int D) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int G>
-int launch_dg(const DecodeLaunch& a) {
+template <int D, int G, int RULE>
+int launch_dgr(const DecodeLaunch& a) {
   using C = DecCfg<D, G>;
-  auto kern = decode_partial_kernel<D, G>;
+  auto kern = decode_partial_kernel<D, G, RULE>;
   static uint64_t attr_done = 0;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
@@ -590,11 +594,23 @@ int launch_dg(const DecodeLaunch& a) {
   kern<<<grid, kDecThreads, C::kSmemBytes, a.stream>>>(
       mk, mv, static_cast<const __nv_bfloat16*>(a.q), a.o_part, a.lse_part, a.skip_mask,
       a.status, a.Hq, a.Hkv, a.L, a.split_len, a.n_splits, a.scale_log2, a.tau_log2,
-      a.tau_is_inf, a.wait_limit_ns, a.withhold_v, a.rule);
+      a.tau_is_inf, a.wait_limit_ns, a.withhold_v);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   decode_combine_kernel<D><<<a.B * a.Hq, D, 0, a.stream>>>(
       a.o_part, a.lse_part, static_cast<__nv_bfloat16*>(a.o), a.n_splits);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D, int G>
+int launch_dg(const DecodeLaunch& a) {
+  switch (a.rule) {
+    case 0: return launch_dgr<D, G, 0>(a);
+    case ATTN_DECODE_RULE_PER_HEAD: return launch_dgr<D, G, ATTN_DECODE_RULE_PER_HEAD>(a);
+    case ATTN_DECODE_RULE_SINK_SEED: return launch_dgr<D, G, ATTN_DECODE_RULE_SINK_SEED>(a);
+    case ATTN_DECODE_RULE_PER_HEAD | ATTN_DECODE_RULE_SINK_SEED:
+      return launch_dgr<D, G, ATTN_DECODE_RULE_PER_HEAD | ATTN_DECODE_RULE_SINK_SEED>(a);
+    default: return ATTN_ERR_INVALID_ARG;
+  }
 }
 
 template <int D>
