@@ -19,7 +19,7 @@ import os
 
 __all__ = [
     "AttnError", "lib", "attn_prefill", "attn_prefill_ex", "attn_decode", "attn_decode_ex",
-    "attn_decode_noalloc", "attn_decode_rule", "RULE_GROUP", "RULE_PER_HEAD", "RULE_SINK_SEED",
+    "attn_decode_noalloc", "attn_decode_rule", "attn_decode_paged", "decode_paged", "RULE_GROUP", "RULE_PER_HEAD", "RULE_SINK_SEED",
     "attn_decode_split_len", "attn_decode_tile", "attn_decode_workspace_bytes",
     "attn_set_stream", "attn_sync_status", "attn_last_timeout_site", "attn_set_wait_limit_ms",
     "attn_test_withhold_copy", "attn_status_string", "attn_shutdown", "prefill", "decode", "STATUS",
@@ -56,6 +56,8 @@ def lib() -> ctypes.CDLL:
         "attn_decode_ex": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, vp, vp, vp, sz]),
         "attn_decode_noalloc": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, vp, vp]),
         "attn_decode_rule": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, ci, vp, vp, vp, sz]),
+        "attn_decode_paged": (ci, [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, cf, ci, vp, vp,
+                                   vp, sz]),
         "attn_decode_split_len": (ci, [ci, ci, ci]),
         "attn_decode_tile": (ci, []),
         "attn_decode_workspace_bytes": (sz, [ci, ci, ci, ci, ci]),
@@ -100,6 +102,14 @@ def attn_decode_rule(q, K, V, o, B, Hq, Hkv, L, d, tau, rule, stream=None, skip_
                      ws_bytes=0) -> int:
     return lib().attn_decode_rule(q, K, V, o, B, Hq, Hkv, L, d, float(tau), int(rule), stream,
                                   skip_mask, ws, ws_bytes)
+
+
+def attn_decode_paged(q, K_pages, V_pages, block_table, seq_lens, o, B, Hq, Hkv, num_pages,
+                      max_pages_per_seq, max_seq_len, d, tau, rule=0, stream=None, skip_mask=None,
+                      ws=None, ws_bytes=0) -> int:
+    return lib().attn_decode_paged(q, K_pages, V_pages, block_table, seq_lens, o, B, Hq, Hkv,
+                                   num_pages, max_pages_per_seq, max_seq_len, d, float(tau),
+                                   int(rule), stream, skip_mask, ws, ws_bytes)
 
 
 def attn_decode_noalloc(q, K, V, o, B, Hq, Hkv, L, d, tau, stream=None, skip_mask=None) -> int:
@@ -210,4 +220,35 @@ def decode(q, K, V, tau: float = math.inf, out=None, skip_mask: bool = False, st
                           tau, rule, _stream_ptr(stream),
                           mask.data_ptr() if mask is not None else None, ws, wsb)
     _check(st, "attn_decode_rule")
+    return (o, mask) if skip_mask else o
+
+
+def decode_paged(q, K_pages, V_pages, block_table, seq_lens, max_seq_len: int, tau: float = math.inf,
+                 out=None, skip_mask: bool = False, stream=None, rule: int = RULE_GROUP):
+    """o = Skip Softmax decode from a paged KV cache.
+
+    q [B,Hq,d]; K_pages/V_pages [num_pages,Hkv,64,d] bf16; block_table int32
+    [B,max_pages]; seq_lens int32 [B]; all CUDA tensors.
+    """
+    import torch
+
+    B, Hq, d = q.shape
+    num_pages, Hkv = K_pages.shape[0], K_pages.shape[1]
+    for t in (q, K_pages, V_pages):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise AttnError(1, "decode_paged (tensors must be contiguous bf16 CUDA tensors)")
+    for t in (block_table, seq_lens):
+        if t.dtype != torch.int32 or not t.is_cuda or not t.is_contiguous():
+            raise AttnError(1, "decode_paged (block_table/seq_lens must be contiguous int32 CUDA tensors)")
+    o = out if out is not None else torch.empty_like(q)
+    mask = None
+    if skip_mask:
+        rows = Hq if rule & RULE_PER_HEAD else Hkv
+        mask = torch.empty(B, rows, -(-max_seq_len // attn_decode_tile()), dtype=torch.uint8,
+                           device=q.device)
+    st = attn_decode_paged(q.data_ptr(), K_pages.data_ptr(), V_pages.data_ptr(), block_table.data_ptr(),
+                           seq_lens.data_ptr(), o.data_ptr(), B, Hq, Hkv, num_pages,
+                           block_table.shape[1], max_seq_len, d, tau, rule, _stream_ptr(stream),
+                           mask.data_ptr() if mask is not None else None)
+    _check(st, "attn_decode_paged")
     return (o, mask) if skip_mask else o

@@ -182,21 +182,16 @@ int attn_decode_ex(const void* q, const void* K, const void* V, void* o, int B, 
                           skip_mask, ws, ws_bytes);
 }
 
-int attn_decode_rule(const void* q, const void* K, const void* V, void* o, int B, int Hq, int Hkv,
-                     int L, int d, float tau, int rule, void* stream, uint8_t* skip_mask, void* ws,
-                     size_t ws_bytes) {
-  if (rule & ~(ATTN_DECODE_RULE_PER_HEAD | ATTN_DECODE_RULE_SINK_SEED)) return ATTN_ERR_INVALID_ARG;
-  int st = check_decode(q, K, V, o, B, Hq, Hkv, L, d, tau);
-  if (st != ATTN_OK) return st;
-  if (ws == nullptr && ws_bytes != 0) return ATTN_ERR_INVALID_ARG;
-  if (ws != nullptr && (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return ATTN_ERR_INVALID_ARG;
-  int dev = 0;
-  int* status = nullptr;
-  if ((st = device_ready(&dev, &status)) != ATTN_OK) return st;
-  const int ls = attn_decode_split_len(B, Hkv, L);
-  const int n_splits = (L + ls - 1) / ls;
+}  // extern "C"
+
+namespace {
+
+// Shared tail of the decode entry points: split layout, workspace, launch.
+int run_decode(bss::DecodeLaunch& a, int dev, void* ws, size_t ws_bytes) {
+  const int ls = attn_decode_split_len(a.B, a.Hkv, a.L);
+  const int n_splits = (a.L + ls - 1) / ls;
   size_t ob = 0, need = 0;
-  decode_ws_layout(B, Hq, n_splits, d, &ob, &need);
+  decode_ws_layout(a.B, a.Hq, n_splits, a.d, &ob, &need);
   if (ws == nullptr) {
     std::lock_guard<std::mutex> lk(g_mu);
     if (g_ws_bytes[dev] < need) {
@@ -214,6 +209,36 @@ int attn_decode_rule(const void* q, const void* K, const void* V, void* o, int B
   } else if (ws_bytes < need) {
     return ATTN_ERR_INVALID_ARG;
   }
+  a.scale_log2 = kLog2e / std::sqrt(static_cast<float>(a.d));
+  a.split_len = ls;
+  a.n_splits = n_splits;
+  a.o_part = static_cast<float*>(ws);
+  a.lse_part = reinterpret_cast<float*>(static_cast<char*>(ws) + ob);
+  a.wait_limit_ns = g_wait_limit_ns;
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    a.withhold_v = g_withhold_v;
+  }
+  return bss::launch_decode(a);
+}
+
+bool rule_ok(int rule) { return (rule & ~(ATTN_DECODE_RULE_PER_HEAD | ATTN_DECODE_RULE_SINK_SEED)) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+int attn_decode_rule(const void* q, const void* K, const void* V, void* o, int B, int Hq, int Hkv,
+                     int L, int d, float tau, int rule, void* stream, uint8_t* skip_mask, void* ws,
+                     size_t ws_bytes) {
+  if (!rule_ok(rule)) return ATTN_ERR_INVALID_ARG;
+  int st = check_decode(q, K, V, o, B, Hq, Hkv, L, d, tau);
+  if (st != ATTN_OK) return st;
+  if (ws == nullptr && ws_bytes != 0) return ATTN_ERR_INVALID_ARG;
+  if (ws != nullptr && (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return ATTN_ERR_INVALID_ARG;
+  int dev = 0;
+  int* status = nullptr;
+  if ((st = device_ready(&dev, &status)) != ATTN_OK) return st;
   bss::DecodeLaunch a{};
   a.q = q;
   a.K = K;
@@ -224,23 +249,56 @@ int attn_decode_rule(const void* q, const void* K, const void* V, void* o, int B
   a.Hkv = Hkv;
   a.L = L;
   a.d = d;
-  a.scale_log2 = kLog2e / std::sqrt(static_cast<float>(d));
   a.tau_is_inf = std::isinf(tau) ? 1 : 0;
   a.tau_log2 = a.tau_is_inf ? 0.f : tau * kLog2e;
-  a.split_len = ls;
-  a.n_splits = n_splits;
-  a.o_part = static_cast<float*>(ws);
-  a.lse_part = reinterpret_cast<float*>(static_cast<char*>(ws) + ob);
   a.skip_mask = skip_mask;
   a.status = status;
-  a.wait_limit_ns = g_wait_limit_ns;
   a.stream = static_cast<cudaStream_t>(stream);
   a.rule = rule;
-  {
-    std::lock_guard<std::mutex> lk(g_mu);
-    a.withhold_v = g_withhold_v;
-  }
-  return bss::launch_decode(a);
+  return run_decode(a, dev, ws, ws_bytes);
+}
+
+int attn_decode_paged(const void* q, const void* K_pages, const void* V_pages,
+                      const int32_t* block_table, const int32_t* seq_lens, void* o, int B, int Hq,
+                      int Hkv, int num_pages, int max_pages_per_seq, int max_seq_len, int d,
+                      float tau, int rule, void* stream, uint8_t* skip_mask, void* ws,
+                      size_t ws_bytes) {
+  if (!rule_ok(rule)) return ATTN_ERR_INVALID_ARG;
+  if (!block_table || !seq_lens) return ATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(block_table) & 3u) || (reinterpret_cast<uintptr_t>(seq_lens) & 3u))
+    return ATTN_ERR_INVALID_ARG;
+  if (num_pages <= 0 || max_pages_per_seq <= 0) return ATTN_ERR_INVALID_ARG;
+  if (static_cast<long long>(num_pages) * Hkv > (1ll << 31) - 1) return ATTN_ERR_UNSUPPORTED;
+  if (max_seq_len > static_cast<long long>(max_pages_per_seq) * bss::kDecodeTile)
+    return ATTN_ERR_INVALID_ARG;
+  int st = check_decode(q, K_pages, V_pages, o, B, Hq, Hkv, max_seq_len, d, tau);
+  if (st != ATTN_OK) return st;
+  if (ws == nullptr && ws_bytes != 0) return ATTN_ERR_INVALID_ARG;
+  if (ws != nullptr && (reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return ATTN_ERR_INVALID_ARG;
+  int dev = 0;
+  int* status = nullptr;
+  if ((st = device_ready(&dev, &status)) != ATTN_OK) return st;
+  bss::DecodeLaunch a{};
+  a.q = q;
+  a.K = K_pages;
+  a.V = V_pages;
+  a.o = o;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.L = max_seq_len;
+  a.d = d;
+  a.tau_is_inf = std::isinf(tau) ? 1 : 0;
+  a.tau_log2 = a.tau_is_inf ? 0.f : tau * kLog2e;
+  a.skip_mask = skip_mask;
+  a.status = status;
+  a.stream = static_cast<cudaStream_t>(stream);
+  a.rule = rule;
+  a.block_table = block_table;
+  a.seq_lens = seq_lens;
+  a.max_pages = max_pages_per_seq;
+  a.num_pages = num_pages;
+  return run_decode(a, dev, ws, ws_bytes);
 }
 
 int attn_decode(const void* q, const void* K, const void* V, void* o, int B, int Hq, int Hkv,

@@ -131,7 +131,7 @@ __device__ __forceinline__ void load_row_floats(const float* p, float (&v)[G]) {
 
 }  // namespace
 
-template <int D, int G, int RULE>
+template <int D, int G, int RULE, bool PAGED>
 __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
     decode_partial_kernel(const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV,
@@ -139,7 +139,9 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
                           float* __restrict__ lse_part, uint8_t* __restrict__ skip_mask,
                           int* __restrict__ status, int Hq, int Hkv, int L, int split_len,
                           int n_splits, float scale_log2, float tau_log2, int tau_is_inf,
-                          unsigned long long wait_limit_ns, int withhold_v) {
+                          unsigned long long wait_limit_ns, int withhold_v,
+                          const int* __restrict__ block_table, const int* __restrict__ seq_lens,
+                          int max_pages) {
   using C = DecCfg<D, G>;
   constexpr unsigned FULL = 0xffffffffu;
   constexpr int kLog2P = ilog2(C::kP);
@@ -170,18 +172,53 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
   const int kv = blockIdx.y;
   const int b = blockIdx.z;
   const int bh = b * Hkv + kv;
-  const int n_tiles_all = (L + kDecodeTile - 1) / kDecodeTile;
-  const int t_begin = split * (split_len / kDecodeTile);
-  const int t_end = min(n_tiles_all, t_begin + split_len / kDecodeTile);
+  // Paged KV cache: L is the longest sequence; this one has Lb keys, clamped
+  // to what its row of the block table can address.
+  int Lb = L;
+  if constexpr (PAGED) Lb = max(0, min(min(seq_lens[b], L), max_pages * kDecodeTile));
+  const int n_tiles_all = (L + kDecodeTile - 1) / kDecodeTile;  // length of a mask row
+  const int n_tiles_b = (Lb + kDecodeTile - 1) / kDecodeTile;
+  const int tps = split_len / kDecodeTile;
+  const int t_begin = split * tps;
+  const int t_end = min(n_tiles_b, t_begin + tps);
   const int nt = t_end - t_begin;
   const float NEG_INF = -__int_as_float(0x7f800000);
 
-  // one tile = kPanels TMA boxes of 64 columns x 64 keys; rows past L read as zeros
+  if constexpr (PAGED) {
+    // tiles of this split past the end of the sequence are not visited
+    if (skip_mask) {
+      const int rows = per_head ? G : 1;
+      for (int idx = tid; idx < rows * tps; idx += kDecThreads) {
+        const int t = t_begin + idx % tps, r = idx / tps;
+        if (t >= n_tiles_b && t < n_tiles_all) {
+          const size_t mrow = per_head ? static_cast<size_t>(b) * Hq + kv * G + r : bh;
+          skip_mask[mrow * n_tiles_all + t] = 2;
+        }
+      }
+    }
+    if (nt <= 0) {  // the whole split lies past the end: zero weight in the merge
+      for (int idx = tid; idx < G * D; idx += kDecThreads) {
+        const size_t row = static_cast<size_t>(b) * Hq + kv * G + idx / D;
+        o_part[(row * n_splits + split) * D + idx % D] = 0.f;
+      }
+      if (tid < G) lse_part[(static_cast<size_t>(b) * Hq + kv * G + tid) * n_splits + split] = NEG_INF;
+      return;
+    }
+  }
+
+  // one tile = kPanels TMA boxes of 64 columns x 64 keys; rows past L read as
+  // zeros.  Paged: tile t of this sequence is page block_table[b][t], whose
+  // 64 keys of KV head kv are row (page * Hkv + kv) of the page pool.
   auto issue = [&](uint32_t dst, const CUtensorMap* map, uint32_t bar, int t) {
     mbar_arrive_expect_tx(bar, C::kTileBytes);
+    int c1 = t * kDecodeTile, c2 = bh;
+    if constexpr (PAGED) {
+      c1 = 0;
+      c2 = block_table[static_cast<size_t>(b) * max_pages + t] * Hkv + kv;
+    }
 #pragma unroll
     for (int p = 0; p < C::kPanels; ++p)
-      tma_load_3d(dst + p * C::kPanelBytes, map, bar, p * 64, t * kDecodeTile, bh);
+      tma_load_3d(dst + p * C::kPanelBytes, map, bar, p * 64, c1, c2);
   };
 
   if (tid == 0) {
@@ -313,7 +350,7 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
     const bool got = mbar_wait(b_seed, 0, never, wait_limit_ns);
     ok = ok && got;
     float sv0[C::kSIters];
-    const float wm0 = tile_scores(smem + C::kOffV, L, sv0);
+    const float wm0 = tile_scores(smem + C::kOffV, Lb, sv0);
     if (kl == 0 && leader) wmax[(kWarps + warp) * G + row_q] = wm0;  // buffer 1; tile 0 uses buffer 0
     __syncthreads();
     const float* wb = wmax + kWarps * G;
@@ -332,7 +369,7 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
       const bool got = mbar_wait(b_k_full(ks), (i / kKStages) & 1, never, wait_limit_ns);
       ok = ok && got;  // on a give-up the scores are garbage and dropped at the barrier
       const uint8_t* kt = smem + C::kOffK + ks * C::kTileBytes;
-      const int key_lim = L - (t_begin + i) * kDecodeTile;  // keys >= key_lim are past L
+      const int key_lim = Lb - (t_begin + i) * kDecodeTile;  // keys >= key_lim are past the end
       const float wm = tile_scores(kt, key_lim, sv);
       if (kl == 0 && leader) wmax[((i & 1) * kWarps + warp) * G + row_q] = wm;
     }
@@ -428,9 +465,14 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
         }
         const uint8_t* vt = smem + C::kOffV + vs * C::kTileBytes;
         const float* pr = p_ring + (t % kPRing) * kDecodeTile * G;
+        // contiguous cache: rows past L arrive as zeros (with p = 0); paged:
+        // rows past the end of the sequence are whatever the page holds and
+        // are left out
+        const int key_lim_v = PAGED ? Lb - (t_begin + t) * kDecodeTile : kDecodeTile;
 #pragma unroll
         for (int e2 = 0; e2 < C::kVKeys; ++e2) {
-          const int key = kg + C::kGroups * e2;  // rows past L are zeros with p = 0
+          const int key = kg + C::kGroups * e2;
+          if (PAGED && key >= key_lim_v) continue;
           const uint4 u = *reinterpret_cast<const uint4*>(vt + chunk_off<D>(key, ch));
           float2 vf[4];
           bf16x8_to_f32(u, vf);
@@ -574,10 +616,10 @@ bool dec_map(CUtensorMap* m, const void* base, int BH, int L, int D) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int G, int RULE>
-int launch_dgr(const DecodeLaunch& a) {
+template <int D, int G, int RULE, bool PAGED>
+int launch_dgrp(const DecodeLaunch& a) {
   using C = DecCfg<D, G>;
-  auto kern = decode_partial_kernel<D, G, RULE>;
+  auto kern = decode_partial_kernel<D, G, RULE, PAGED>;
   static uint64_t attr_done = 0;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
@@ -588,17 +630,27 @@ int launch_dgr(const DecodeLaunch& a) {
     attr_done |= uint64_t(1) << dev;
   }
   CUtensorMap mk, mv;
-  if (!dec_map(&mk, a.K, a.B * a.Hkv, a.L, D) || !dec_map(&mv, a.V, a.B * a.Hkv, a.L, D))
+  if (PAGED) {  // the page pool as [num_pages * Hkv, 64, D]
+    if (!dec_map(&mk, a.K, a.num_pages * a.Hkv, kDecodeTile, D) ||
+        !dec_map(&mv, a.V, a.num_pages * a.Hkv, kDecodeTile, D))
+      return ATTN_ERR_CUDA;
+  } else if (!dec_map(&mk, a.K, a.B * a.Hkv, a.L, D) || !dec_map(&mv, a.V, a.B * a.Hkv, a.L, D)) {
     return ATTN_ERR_CUDA;
+  }
   dim3 grid(a.n_splits, a.Hkv, a.B);
   kern<<<grid, kDecThreads, C::kSmemBytes, a.stream>>>(
       mk, mv, static_cast<const __nv_bfloat16*>(a.q), a.o_part, a.lse_part, a.skip_mask,
       a.status, a.Hq, a.Hkv, a.L, a.split_len, a.n_splits, a.scale_log2, a.tau_log2,
-      a.tau_is_inf, a.wait_limit_ns, a.withhold_v);
+      a.tau_is_inf, a.wait_limit_ns, a.withhold_v, a.block_table, a.seq_lens, a.max_pages);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   decode_combine_kernel<D><<<a.B * a.Hq, D, 0, a.stream>>>(
       a.o_part, a.lse_part, static_cast<__nv_bfloat16*>(a.o), a.n_splits);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D, int G, int RULE>
+int launch_dgr(const DecodeLaunch& a) {
+  return a.block_table ? launch_dgrp<D, G, RULE, true>(a) : launch_dgrp<D, G, RULE, false>(a);
 }
 
 template <int D, int G>

@@ -49,6 +49,13 @@ struct DecodeLaunch {
   cudaStream_t stream;
   int withhold_v;  // test support: 1 = every CTA withholds its first V copy
   int rule;        // ATTN_DECODE_RULE_* bits
+  // paged KV cache (block_table == nullptr: contiguous [B, Hkv, L, d]); then
+  // K and V are page pools [num_pages, Hkv, 64, d] and L is the longest
+  // sequence
+  const int* block_table;  // [B, max_pages] page ids
+  const int* seq_lens;     // [B] keys per sequence
+  int max_pages;
+  int num_pages;
 };
 
 int launch_decode(const DecodeLaunch& a);

@@ -134,6 +134,33 @@ ATTN_API int attn_decode_rule(const void* q, const void* K, const void* V, void*
                               uint8_t* skip_mask, void* ws, size_t ws_bytes);
 
 /*
+ * Decode from a paged KV cache (the layout serving engines keep: fixed-size
+ * pages in one pool, a per-sequence table of page ids, ragged lengths).
+ *   K_pages, V_pages  page pools, bf16 [num_pages, Hkv, 64, d]: page p holds
+ *                     64 consecutive keys of every KV head of one sequence.
+ *   block_table       device int32 [B, max_pages_per_seq]: entry (b, t) is the
+ *                     page holding keys [64 t, 64 t + 64) of sequence b.
+ *                     Only entries t < ceil(len_b / 64) are read.
+ *   seq_lens          device int32 [B]: len_b, the keys of sequence b; used as
+ *                     min(len_b, max_seq_len).  len_b must be >= 1 (a row with
+ *                     no key has no softmax; its output is NaN).
+ *   max_seq_len       the longest sequence (<= 64 * max_pages_per_seq); the
+ *                     split layout is that of attn_decode_ex with L = max_seq_len.
+ *   Keys past len_b inside the last page may hold anything (NaN included);
+ *   they are masked.  A page id outside [0, num_pages) reads zeros (no fault).
+ *   skip_mask (nullable): [B, Hkv, ceil(max_seq_len/64)], or [B, Hq, ...] with
+ *   ATTN_DECODE_RULE_PER_HEAD; tiles past len_b are marked 2 (not visited).
+ *   Other arguments and errors as attn_decode_rule; ATTN_ERR_INVALID_ARG also
+ *   for null or unaligned block_table / seq_lens, num_pages or
+ *   max_pages_per_seq <= 0, and max_seq_len > 64 * max_pages_per_seq.
+ */
+ATTN_API int attn_decode_paged(const void* q, const void* K_pages, const void* V_pages,
+                               const int32_t* block_table, const int32_t* seq_lens, void* o, int B,
+                               int Hq, int Hkv, int num_pages, int max_pages_per_seq,
+                               int max_seq_len, int d, float tau, int rule, void* stream,
+                               uint8_t* skip_mask, void* ws, size_t ws_bytes);
+
+/*
  * Decode that allocates nothing, for callers that cannot allocate device
  * memory (a serving engine that has reserved all of HBM for its own pools, a
  * latency-critical loop that must not meet the implicit synchronisation of
