@@ -18,7 +18,7 @@ import math
 import os
 
 __all__ = [
-    "AttnError", "lib", "attn_prefill", "attn_prefill_ex", "attn_decode", "attn_decode_ex",
+    "AttnError", "lib", "attn_prefill", "attn_prefill_ex", "attn_prefill_host", "prefill_host", "attn_decode", "attn_decode_ex",
     "attn_decode_noalloc", "attn_decode_rule", "attn_decode_paged", "decode_paged", "RULE_GROUP", "RULE_PER_HEAD", "RULE_SINK_SEED",
     "attn_decode_split_len", "attn_decode_tile", "attn_decode_workspace_bytes",
     "attn_set_stream", "attn_sync_status", "attn_last_timeout_site", "attn_set_wait_limit_ms",
@@ -52,6 +52,7 @@ def lib() -> ctypes.CDLL:
     sig = {
         "attn_prefill": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, ci]),
         "attn_prefill_ex": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, ci, vp, vp]),
+        "attn_prefill_host": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, ci, ci, vp]),
         "attn_decode": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf]),
         "attn_decode_ex": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, vp, vp, vp, sz]),
         "attn_decode_noalloc": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, vp, vp]),
@@ -85,6 +86,11 @@ def attn_prefill(Q, K, V, O, B, Hq, Hkv, N, d, causal, tau, Br, Bc) -> int:
 def attn_prefill_ex(Q, K, V, O, B, Hq, Hkv, N, d, causal, tau, Br, Bc, stream=None, skip_mask=None) -> int:
     return lib().attn_prefill_ex(Q, K, V, O, B, Hq, Hkv, N, d, int(causal), float(tau), Br, Bc,
                                  stream, skip_mask)
+
+
+def attn_prefill_host(Qh, Kh, Vh, Oh, B, Hq, Hkv, N, d, causal, tau, Br, Bc, chunk=0, stream=None) -> int:
+    return lib().attn_prefill_host(Qh, Kh, Vh, Oh, B, Hq, Hkv, N, d, int(causal), float(tau), Br, Bc,
+                                   int(chunk), stream)
 
 
 def attn_decode(q, K, V, o, B, Hq, Hkv, L, d, tau) -> int:
@@ -194,6 +200,25 @@ def prefill(Q, K, V, causal: bool, tau: float = math.inf, Br: int = 128, Bc: int
                          mask.data_ptr() if mask is not None else None)
     _check(st, "attn_prefill_ex")
     return (O, mask) if skip_mask else O
+
+
+def prefill_host(Qh, Kh, Vh, causal: bool, tau: float = math.inf, Br: int = 128, Bc: int = 128,
+                 out=None, chunk: int = 0, stream=None):
+    """attn_prefill_host on host (CPU) bf16 tensors; pinned memory lets the
+    copies overlap.  Asynchronous on ``stream``: synchronise it before reading
+    the returned tensor."""
+    import torch
+
+    B, Hq, N, d = Qh.shape
+    Hkv = Kh.shape[1]
+    for t in (Qh, Kh, Vh):
+        if t.dtype != torch.bfloat16 or t.is_cuda or not t.is_contiguous():
+            raise AttnError(1, "prefill_host (tensors must be contiguous bf16 host tensors)")
+    Oh = out if out is not None else torch.empty_like(Qh, pin_memory=Qh.is_pinned())
+    st = attn_prefill_host(Qh.data_ptr(), Kh.data_ptr(), Vh.data_ptr(), Oh.data_ptr(), B, Hq, Hkv, N, d,
+                           causal, tau, Br, Bc, chunk, _stream_ptr(stream))
+    _check(st, "attn_prefill_host")
+    return Oh
 
 
 def decode(q, K, V, tau: float = math.inf, out=None, skip_mask: bool = False, stream=None,

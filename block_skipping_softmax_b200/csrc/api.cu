@@ -95,6 +95,7 @@ void decode_ws_layout(int B, int Hq, int n_splits, int d, size_t* o_bytes, size_
 }  // namespace
 
 namespace bss {
+void host_pipeline_release();  // host_pipeline.cu
 // Current device (sm_100 checked) and its device status word, for entry
 // points defined in other files.
 int device_context(int* dev, int** status) { return device_ready(dev, status); }
@@ -361,6 +362,7 @@ const char* attn_status_string(int s) {
 }
 
 void attn_shutdown(void) {
+  bss::host_pipeline_release();
   std::lock_guard<std::mutex> lk(g_mu);
   int cur = 0;
   const bool have = cudaGetDevice(&cur) == cudaSuccess;

@@ -81,6 +81,28 @@ ATTN_API int attn_prefill_ex(const void* Q, const void* K, const void* V, void* 
                     uint8_t* skip_mask);
 
 /*
+ * Prefill with the inputs and the output in host memory: the batch is cut
+ * into chunks of `chunk` sequences (0: B/8 rounded up) that flow through two
+ * library-owned device buffer sets on two library streams, so the copy of
+ * one chunk to the device overlaps the kernel and the copy back of the
+ * previous one.  Qh, Kh, Vh, Oh are host pointers with the layouts of
+ * attn_prefill; page-locked (pinned) memory is needed for the copies to
+ * overlap.  The call is asynchronous and ordered on `stream` (cudaStream_t as
+ * void*, NULL = legacy stream) like a kernel launch: work queued on `stream`
+ * before the call happens before it, and Oh is complete once `stream`
+ * reaches the point after the call (e.g. after cudaStreamSynchronize).  The
+ * host buffers must stay valid and unmodified until then.  One call at a
+ * time per process (calls from several host threads are serialised, their
+ * device work may overlap only through their own streams' order).  The
+ * device buffers (about 2 chunks of Q, K, V and O) are kept for the next call
+ * and freed by attn_shutdown().  Errors: as attn_prefill, plus
+ * ATTN_ERR_INVALID_ARG for null host pointers or chunk < 0.
+ */
+ATTN_API int attn_prefill_host(const void* Qh, const void* Kh, const void* Vh, void* Oh, int B,
+                               int Hq, int Hkv, int N, int d, int causal, float tau, int Br, int Bc,
+                               int chunk, void* stream);
+
+/*
  * Decode: one new query token per (batch, query head) against L cached keys,
  * no mask.  The rows of the skip test are the g = Hq/Hkv query heads that
  * share one KV head (they share the V tile that a skip avoids loading).  The
