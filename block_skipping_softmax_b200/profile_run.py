@@ -1,0 +1,51 @@
+"""Run one named workload's kernel a few times, for a profiler to capture.
+
+    python -m block_skipping_softmax_b200.profile_run --workload llama3_8b_causal_N8192 \
+        --tau inf --launches 3
+
+Inputs follow the workload's recipe (drawn on the GPU, as in bench.py); no
+timing is printed, since numbers taken under a profiler are not
+measurements.  The process exits non-zero if a kernel reports a status.
+"""
+from __future__ import annotations
+
+import argparse
+import math
+import sys
+
+
+def main(argv=None) -> int:
+    import torch
+
+    import block_skipping_softmax_b200 as bss
+    from block_skipping_softmax_b200 import inputs
+
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--workload", required=True, choices=sorted(inputs.WORKLOADS))
+    ap.add_argument("--tau", default="inf")
+    ap.add_argument("--launches", type=int, default=3)
+    args = ap.parse_args(argv)
+    tau = math.inf if args.tau == "inf" else float(args.tau)
+    w = inputs.WORKLOADS[args.workload]
+    dev = torch.device("cuda", 0)
+    if w["kind"] == "prefill":
+        Q, K, V = inputs.prefill_inputs(w["B"], w["Hq"], w["Hkv"], w["N"], w["d"], seed=0,
+                                        device=str(dev), **w["gen"])
+        O = torch.empty_like(Q)
+        for _ in range(args.launches):
+            bss.prefill(Q, K, V, w["causal"], tau, w["Br"], w["Bc"], out=O)
+    else:
+        q, K, V = inputs.decode_inputs(w["B"], w["Hq"], w["Hkv"], w["L"], w["d"], seed=0, **w["gen"])
+        q, K, V = q.to(dev), K.to(dev), V.to(dev)
+        o = torch.empty_like(q)
+        for _ in range(args.launches):
+            bss.decode(q, K, V, tau, out=o)
+    st = bss.attn_sync_status()
+    if st != 0:
+        print(f"kernel status {bss.attn_status_string(st)}", file=sys.stderr)
+        return 1
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())
