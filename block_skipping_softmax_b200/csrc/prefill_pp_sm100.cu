@@ -230,6 +230,17 @@ __global__ void __launch_bounds__(kPPThreads, 1)
   const int g = Hq / Hkv;
   const int n_tiles = (N + BC - 1) / BC;
   const long long n_items = static_cast<long long>(BH) * n_pairs;
+  // The k-th work item of this CTA: items go out in rounds of gridDim.x.
+  // Causal items are numbered longest first and go out in a "snake": CTAs in
+  // ascending order in even rounds and descending in odd ones, which evens
+  // out the work per CTA (for the causal 8B layer the busiest CTA had 14 %
+  // more than the mean with plain round robin, 1.6 % with the snake).
+  // Non-causal items are all equal and keep plain round robin.  Once an index
+  // passes n_items every later one does too.
+  auto item_idx = [&](long long k) -> long long {
+    const long long G = gridDim.x;
+    return k * G + ((CAUSAL && (k & 1)) ? G - 1 - blockIdx.x : blockIdx.x);
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kKS; ++s) mbar_init(b_k_full(s), 1);
@@ -271,7 +282,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       Pending3 pend;
       pend.init();
       bool alive = true;
-      for (long long idx = blockIdx.x; alive && idx < n_items; idx += gridDim.x, ++items) {
+      for (long long idx = item_idx(items); alive && idx < n_items; idx = item_idx(++items)) {
         const Item it = make_item<BC, CAUSAL>(idx, BH, n_pairs, n_rb, N);
         const int bkv = (it.bh / Hq) * Hkv + (it.bh % Hq) / g;
         const int qs = items % C::kQS;
@@ -323,7 +334,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       Pending3 pend;
       pend.init();
       bool alive = true;
-      for (long long idx = blockIdx.x; alive && idx < n_items; idx += gridDim.x) {
+      for (long long k = 0, idx = item_idx(0); alive && idx < n_items; idx = item_idx(++k)) {
         const Item it = make_item<BC, CAUSAL>(idx, BH, n_pairs, n_rb, N);
         const int bkv = (it.bh / Hq) * Hkv + (it.bh % Hq) / g;
         const int T[2] = {it.T0, it.T1};
@@ -415,7 +426,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         mma_commit(b_cm(t, cmc[t]));
         ++cmc[t];
       };
-      for (long long idx = blockIdx.x; alive && idx < n_items; idx += gridDim.x, ++items) {
+      for (long long idx = item_idx(items); alive && idx < n_items; idx = item_idx(++items)) {
         const Item it = make_item<BC, CAUSAL>(idx, BH, n_pairs, n_rb, N);
         const int T[2] = {it.T0, it.T1};
         const int qs = items % C::kQS;
@@ -528,7 +539,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       }
     };
     bool ok = true, failed = false;
-    for (long long idx = blockIdx.x; ok && idx < n_items; idx += gridDim.x) {
+    for (long long k = 0, idx = item_idx(0); ok && idx < n_items; idx = item_idx(++k)) {
       const Item it = make_item<BC, CAUSAL>(idx, BH, n_pairs, n_rb, N);
       const int T = t == 0 ? it.T0 : it.T1;
       const int qs = items % C::kQS;
