@@ -387,6 +387,10 @@ def main():
             "ms": ms_x, "dense_tflops": f / (ms_x * 1e-3) / 1e12,
             "executed_tflops": executed / (ms_x * 1e-3) / 1e12,
             "frac_of_peak": f / (ms_x * 1e-3) / 1e12 / peaks["bf16_tflops"],
+            # a launch of 50 ms or more runs under the power cap: compare it
+            # with the sustained GEMM figure as well
+            "frac_of_sustained_peak": (f / (ms_x * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"]
+                                       if ms_x >= 50.0 else None),
             "skipped_fraction": skipped, "tiles_visited": visited}
 
     prefill_extra(MAIN, w, Q, K, V, math.inf, 3, 1)
