@@ -18,7 +18,8 @@ import math
 import os
 
 __all__ = [
-    "AttnError", "lib", "attn_prefill", "attn_prefill_ex", "attn_prefill_host", "prefill_host", "attn_decode", "attn_decode_ex",
+    "AttnError", "lib", "attn_prefill", "attn_prefill_ex", "attn_prefill_host", "prefill_host",
+    "attn_prefill_varlen", "prefill_varlen", "attn_decode", "attn_decode_ex",
     "attn_decode_noalloc", "attn_decode_rule", "attn_decode_paged", "decode_paged", "RULE_GROUP", "RULE_PER_HEAD", "RULE_SINK_SEED",
     "attn_decode_split_len", "attn_decode_tile", "attn_decode_workspace_bytes",
     "attn_set_stream", "attn_sync_status", "attn_last_timeout_site", "attn_set_wait_limit_ms",
@@ -53,6 +54,7 @@ def lib() -> ctypes.CDLL:
         "attn_prefill": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, ci]),
         "attn_prefill_ex": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, ci, vp, vp]),
         "attn_prefill_host": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, ci, ci, vp]),
+        "attn_prefill_varlen": (ci, [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, cf, ci, ci, vp, vp]),
         "attn_decode": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf]),
         "attn_decode_ex": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, vp, vp, vp, sz]),
         "attn_decode_noalloc": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, vp, vp]),
@@ -71,7 +73,10 @@ def lib() -> ctypes.CDLL:
         "attn_shutdown": (None, []),
     }
     for name, (res, args) in sig.items():
-        f = getattr(L, name)
+        try:
+            f = getattr(L, name)
+        except AttributeError:  # an older build: the entry point raises when called
+            continue
         f.restype, f.argtypes = res, args
     _lib = L
     return L
@@ -91,6 +96,12 @@ def attn_prefill_ex(Q, K, V, O, B, Hq, Hkv, N, d, causal, tau, Br, Bc, stream=No
 def attn_prefill_host(Qh, Kh, Vh, Oh, B, Hq, Hkv, N, d, causal, tau, Br, Bc, chunk=0, stream=None) -> int:
     return lib().attn_prefill_host(Qh, Kh, Vh, Oh, B, Hq, Hkv, N, d, int(causal), float(tau), Br, Bc,
                                    int(chunk), stream)
+
+
+def attn_prefill_varlen(Q, K, V, O, cu_seqlens, B, max_seqlen, total_tokens, Hq, Hkv, d, causal, tau,
+                        Br, Bc, stream=None, skip_mask=None) -> int:
+    return lib().attn_prefill_varlen(Q, K, V, O, cu_seqlens, B, max_seqlen, total_tokens, Hq, Hkv, d,
+                                     int(causal), float(tau), Br, Bc, stream, skip_mask)
 
 
 def attn_decode(q, K, V, o, B, Hq, Hkv, L, d, tau) -> int:
@@ -199,6 +210,32 @@ def prefill(Q, K, V, causal: bool, tau: float = math.inf, Br: int = 128, Bc: int
                          causal, tau, Br, Bc, _stream_ptr(stream),
                          mask.data_ptr() if mask is not None else None)
     _check(st, "attn_prefill_ex")
+    return (O, mask) if skip_mask else O
+
+
+def prefill_varlen(Q, K, V, cu_seqlens, max_seqlen: int, causal: bool, tau: float = math.inf,
+                   Br: int = 128, Bc: int = 128, out=None, skip_mask: bool = False, stream=None):
+    """Packed variable-length prefill: Q [total, Hq, d], K/V [total, Hkv, d]
+    bf16 CUDA tensors; cu_seqlens int32 CUDA tensor [B + 1]."""
+    import torch
+
+    total, Hq, d = Q.shape
+    Hkv = K.shape[1]
+    B = cu_seqlens.numel() - 1
+    for t in (Q, K, V):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise AttnError(1, "prefill_varlen (tensors must be contiguous bf16 CUDA tensors)")
+    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda:
+        raise AttnError(1, "prefill_varlen (cu_seqlens must be an int32 CUDA tensor)")
+    O = out if out is not None else torch.empty_like(Q)
+    mask = None
+    if skip_mask:
+        mask = torch.empty(B, Hq, -(-max_seqlen // Br), -(-max_seqlen // Bc), dtype=torch.uint8,
+                           device=Q.device)
+    st = attn_prefill_varlen(Q.data_ptr(), K.data_ptr(), V.data_ptr(), O.data_ptr(), cu_seqlens.data_ptr(),
+                             B, max_seqlen, total, Hq, Hkv, d, causal, tau, Br, Bc, _stream_ptr(stream),
+                             mask.data_ptr() if mask is not None else None)
+    _check(st, "attn_prefill_varlen")
     return (O, mask) if skip_mask else O
 
 

@@ -23,6 +23,11 @@ struct PrefillLaunch {
   int* status;
   unsigned long long wait_limit_ns;
   cudaStream_t stream;
+  // variable-length batch (cu_seqlens != nullptr): Q, O [total, Hq, d] and
+  // K, V [total, Hkv, d]; sequence b is tokens [cu_seqlens[b], cu_seqlens[b+1])
+  // and N is the longest sequence
+  const int* cu_seqlens;
+  int total;
 };
 
 int launch_prefill(const PrefillLaunch& a);     // one row block per CTA (any Br)

@@ -127,29 +127,57 @@ __device__ __forceinline__ void pp_give_up(PPMisc* m, int* status, int where) {
 
 // Work item -> (bh, pair).  Causal: longest pairs first, heads fastest.
 // Non-causal: pairs fastest, so CTAs reading one head's K/V run together.
+// Variable-length batches (VARLEN): N is the longest sequence; items run
+// over (pair, sequence, head), longest pairs first, and a pair past the end
+// of its sequence is an empty item (T0 = 0) that every role skips.
 struct Item {
   int bh, rb0, T0, T1, Tmax;  // T1 = 0 when the second row block does not exist
+  int len, tok0;              // keys of this sequence, and its first token (VARLEN)
 };
 
-template <int BC, bool CAUSAL>
-__device__ __forceinline__ Item make_item(long long idx, int BH, int n_pairs, int n_rb, int N) {
+template <int BC, bool CAUSAL, bool VARLEN>
+__device__ __forceinline__ Item make_item(long long idx, int BH, int n_pairs, int n_rb, int N,
+                                          int Hq, const int* cu_seqlens, int total) {
   Item it;
   int pair;
-  if (CAUSAL) {
+  if (VARLEN) {
     pair = n_pairs - 1 - static_cast<int>(idx / BH);
     it.bh = static_cast<int>(idx % BH);
+    const int b = it.bh / Hq;
+    // clamped, so that a malformed cu_seqlens cannot move a row past the tensors
+    it.tok0 = min(max(cu_seqlens[b], 0), total);
+    it.len = max(0, min(min(N, cu_seqlens[b + 1] - it.tok0), total - it.tok0));
+  } else if (CAUSAL) {
+    pair = n_pairs - 1 - static_cast<int>(idx / BH);
+    it.bh = static_cast<int>(idx % BH);
+    it.len = N;
+    it.tok0 = 0;
   } else {
     pair = static_cast<int>(idx % n_pairs);
     it.bh = static_cast<int>(idx / n_pairs);
+    it.len = N;
+    it.tok0 = 0;
   }
   it.rb0 = 2 * pair;
-  const int n_tiles = (N + BC - 1) / BC;
-  auto visited = [&](int rb) {
-    const int last = min(N, (rb + 1) * kRows) - 1;
-    return CAUSAL ? (last / BC + 1) : n_tiles;
-  };
-  it.T0 = visited(it.rb0);
-  it.T1 = (it.rb0 + 1 < n_rb) ? visited(it.rb0 + 1) : 0;
+  if constexpr (VARLEN) {
+    const int n_tiles = (it.len + BC - 1) / BC;
+    const int n_rb_s = (it.len + kRows - 1) / kRows;
+    auto visited = [&](int rb) {
+      if (rb >= n_rb_s) return 0;
+      const int last = min(it.len, (rb + 1) * kRows) - 1;
+      return CAUSAL ? (last / BC + 1) : n_tiles;
+    };
+    it.T0 = visited(it.rb0);
+    it.T1 = visited(it.rb0 + 1);
+  } else {
+    const int n_tiles = (N + BC - 1) / BC;
+    auto visited = [&](int rb) {
+      const int last = min(N, (rb + 1) * kRows) - 1;
+      return CAUSAL ? (last / BC + 1) : n_tiles;
+    };
+    it.T0 = visited(it.rb0);
+    it.T1 = (it.rb0 + 1 < n_rb) ? visited(it.rb0 + 1) : 0;
+  }
   it.Tmax = max(it.T0, it.T1);
   return it;
 }
@@ -180,15 +208,19 @@ struct Pending3 {
 
 }  // namespace
 
-template <int D, int BC, bool CAUSAL>
+template <int D, int BC, bool CAUSAL, bool VARLEN>
 __global__ void __launch_bounds__(kPPThreads, 1)
     prefill_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                       __nv_bfloat16* __restrict__ O,
                       uint8_t* __restrict__ skip_mask, int* __restrict__ status, int B, int Hq,
                       int Hkv, int N, float scale_log2, float tau_log2, int tau_is_inf,
-                      unsigned long long wait_limit_ns) {
+                      unsigned long long wait_limit_ns, const int* __restrict__ cu_seqlens,
+                      int total) {
   using C = PPCfg<D, BC>;
+  // variable-length batches store O row by row: a TMA store of the last row
+  // block would write into the next sequence's rows
+  constexpr bool kTmaEpi = C::kTmaEpi && !VARLEN;
   constexpr int SB = C::kSB;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -252,7 +284,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
     }
     for (int s = 0; s < C::kQS; ++s) {
       mbar_init(b_q_full(s), 1);
-      mbar_init(b_q_empty(s), C::kTmaEpi ? 2 : 1);  // one arrival per row block's O store
+      mbar_init(b_q_empty(s), kTmaEpi ? 2 : 1);  // one arrival per row block's O store
     }
     mbar_init(b_mma_done, 1);
     for (int t = 0; t < 2; ++t)
@@ -282,8 +314,10 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       Pending3 pend;
       pend.init();
       bool alive = true;
-      for (long long idx = item_idx(items); alive && idx < n_items; idx = item_idx(++items)) {
-        const Item it = make_item<BC, CAUSAL>(idx, BH, n_pairs, n_rb, N);
+      // items counts the non-empty work items (their Q slots); k every index
+      for (long long k = 0, idx = item_idx(0); alive && idx < n_items; idx = item_idx(++k)) {
+        const Item it = make_item<BC, CAUSAL, VARLEN>(idx, BH, n_pairs, n_rb, N, Hq, cu_seqlens, total);
+        if (VARLEN && it.T0 == 0) continue;  // a pair past the end of its sequence
         const int bkv = (it.bh / Hq) * Hkv + (it.bh % Hq) / g;
         const int qs = items % C::kQS;
         if (items >= C::kQS && !mbar_wait(b_q_empty(qs), ((items / C::kQS) - 1) & 1, abort_flag,
@@ -295,8 +329,12 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         mbar_arrive_expect_tx(b_q_full(qs), nq * C::kQTile);
         for (int t = 0; t < nq; ++t)
           for (int p = 0; p < C::kPanels; ++p)
-            tma_load_3d(sQ + qs * C::kQSlot + t * C::kQTile + p * C::kQPanel, &tmQ, b_q_full(qs),
-                        p * 64, (it.rb0 + t) * kRows, it.bh);
+            if constexpr (VARLEN)  // Q as [tokens, Hq, d]
+              tma_load_3d(sQ + qs * C::kQSlot + t * C::kQTile + p * C::kQPanel, &tmQ, b_q_full(qs),
+                          p * 64, it.bh % Hq, it.tok0 + (it.rb0 + t) * kRows);
+            else
+              tma_load_3d(sQ + qs * C::kQSlot + t * C::kQTile + p * C::kQPanel, &tmQ, b_q_full(qs),
+                          p * 64, (it.rb0 + t) * kRows, it.bh);
         for (int j = 0; j < it.Tmax; ++j) {
           const int s = kload % C::kKS;
           if (pend.n == C::kKS) {  // the slot's previous tile: its S MMAs must have run
@@ -308,9 +346,14 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             pend.pop();
           }
           mbar_arrive_expect_tx(b_k_full(s), C::kKVBytes);
-          for (int p = 0; p < C::kPanels; ++p)
-            tma_load_3d(sK + s * C::kKVBytes + p * C::kKVPanel, &tmK, b_k_full(s), p * 64, j * BC,
-                        bkv);
+          for (int p = 0; p < C::kPanels; ++p) {
+            if constexpr (VARLEN)  // K as [tokens, Hkv, d]
+              tma_load_3d(sK + s * C::kKVBytes + p * C::kKVPanel, &tmK, b_k_full(s), p * 64,
+                          (it.bh % Hq) / g, it.tok0 + j * BC);
+            else
+              tma_load_3d(sK + s * C::kKVBytes + p * C::kKVPanel, &tmK, b_k_full(s), p * 64, j * BC,
+                          bkv);
+          }
           // K tile j is read by S of row block 1 last (if it exists, T1 >= T0)
           if (j < it.T1) pend.push(1, base1 + j, 0);
           else pend.push(0, base0 + j, 0);
@@ -319,6 +362,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         base0 += commits_of<SB>(it.T0);
         base1 += commits_of<SB>(it.T1);
         kdone = items + 1;
+        ++items;
       }
       // never leave with a copy in flight
       for (int i = max(0, kdone - C::kQS); i < kdone; ++i)
@@ -335,7 +379,8 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       pend.init();
       bool alive = true;
       for (long long k = 0, idx = item_idx(0); alive && idx < n_items; idx = item_idx(++k)) {
-        const Item it = make_item<BC, CAUSAL>(idx, BH, n_pairs, n_rb, N);
+        const Item it = make_item<BC, CAUSAL, VARLEN>(idx, BH, n_pairs, n_rb, N, Hq, cu_seqlens, total);
+        if (VARLEN && it.T0 == 0) continue;  // a pair past the end of its sequence
         const int bkv = (it.bh / Hq) * Hkv + (it.bh % Hq) / g;
         const int T[2] = {it.T0, it.T1};
         auto issue_v = [&](int j) -> bool {
@@ -352,9 +397,14 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           }
           const int s = vload % C::kVS;
           mbar_arrive_expect_tx(b_v_full(s), C::kKVBytes);
-          for (int p = 0; p < C::kPanels; ++p)
-            tma_load_3d(sV + s * C::kKVBytes + p * C::kKVPanel, &tmV, b_v_full(s), p * 64, j * BC,
-                        bkv);
+          for (int p = 0; p < C::kPanels; ++p) {
+            if constexpr (VARLEN)  // V as [tokens, Hkv, d]
+              tma_load_3d(sV + s * C::kKVBytes + p * C::kKVPanel, &tmV, b_v_full(s), p * 64,
+                          (it.bh % Hq) / g, it.tok0 + j * BC);
+            else
+              tma_load_3d(sV + s * C::kKVBytes + p * C::kKVPanel, &tmV, b_v_full(s), p * 64, j * BC,
+                          bkv);
+          }
           // P*V of tile j, row block 1 (if it visits j) is issued after row block 0's
           if (j < it.T1) pend.push(1, base1 + min(SB, it.T1) + j, gbase + j);
           else pend.push(0, base0 + min(SB, it.T0) + j, gbase + j);
@@ -426,8 +476,9 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         mma_commit(b_cm(t, cmc[t]));
         ++cmc[t];
       };
-      for (long long idx = item_idx(items); alive && idx < n_items; idx = item_idx(++items)) {
-        const Item it = make_item<BC, CAUSAL>(idx, BH, n_pairs, n_rb, N);
+      for (long long k = 0, idx = item_idx(0); alive && idx < n_items; idx = item_idx(++k)) {
+        const Item it = make_item<BC, CAUSAL, VARLEN>(idx, BH, n_pairs, n_rb, N, Hq, cu_seqlens, total);
+        if (VARLEN && it.T0 == 0) continue;  // a pair past the end of its sequence
         const int T[2] = {it.T0, it.T1};
         const int qs = items % C::kQS;
         dQ = sw128_desc_lo(sQ + qs * C::kQSlot, 16);
@@ -454,7 +505,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         }
         if (!alive) break;
         // the Q slot is free once the item's last S MMA has run
-        if (!C::kTmaEpi && it.Tmax <= SB) mma_commit(b_q_empty(qs));
+        if (!kTmaEpi && it.Tmax <= SB) mma_commit(b_q_empty(qs));
         bool started[2] = {false, false};
         for (int j = 0; alive && j < it.Tmax; ++j) {
           bool v_used = false, k_next = false;
@@ -509,8 +560,9 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           }
           if (k_next) ++kuse;
           if (v_used) ++vuse;
-          if (!C::kTmaEpi && j + SB + 1 == it.Tmax) mma_commit(b_q_empty(qs));  // last S MMAs issued
+          if (!kTmaEpi && j + SB + 1 == it.Tmax) mma_commit(b_q_empty(qs));  // last S MMAs issued
         }
+        ++items;
       }
       // all issued MMAs must finish before TMEM is released
       mma_commit(b_mma_done);
@@ -532,7 +584,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
     // many arrivals on that slot's q_empty the store stands for
     int pend_slot = -1, pend_n = 0;
     auto release_pending = [&]() {
-      if (C::kTmaEpi && pend_slot >= 0) {
+      if (kTmaEpi && pend_slot >= 0) {
         bulk_wait_read_all();
         for (int k = 0; k < pend_n; ++k) mbar_arrive(b_q_empty(pend_slot));
         pend_slot = -1;
@@ -540,7 +592,8 @@ __global__ void __launch_bounds__(kPPThreads, 1)
     };
     bool ok = true, failed = false;
     for (long long k = 0, idx = item_idx(0); ok && idx < n_items; idx = item_idx(++k)) {
-      const Item it = make_item<BC, CAUSAL>(idx, BH, n_pairs, n_rb, N);
+      const Item it = make_item<BC, CAUSAL, VARLEN>(idx, BH, n_pairs, n_rb, N, Hq, cu_seqlens, total);
+      if (VARLEN && it.T0 == 0) continue;  // a pair past the end of its sequence: not a work item
       const int T = t == 0 ? it.T0 : it.T1;
       const int qs = items % C::kQS;
       ++items;
@@ -551,7 +604,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       const int pro = min(SB, T);
       const int rb = it.rb0 + t;
       const int q_idx = rb * kRows + row;
-      const bool row_valid = q_idx < N;
+      const bool row_valid = q_idx < it.len;
       const size_t mask_base =
           skip_mask ? ((static_cast<size_t>(it.bh) * n_rb + rb) * n_tiles) : 0;
       float m_exact = NEG_INF, m_ref = NEG_INF, l_sum = 0.f;
@@ -570,7 +623,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           // last visible column of this row in tile j (-1: none); one integer
           // limit keeps the masking to a compare-select per column
           const int key0 = j * BC;
-          int lim = min(BC - 1, N - 1 - key0);
+          int lim = min(BC - 1, it.len - 1 - key0);
           if (CAUSAL) lim = min(lim, q_idx - key0);
           if (!row_valid) lim = -1;
           if (lim < BC - 1) {
@@ -740,7 +793,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       }
       tc_fence_after();
       const float inv_l = row_valid ? 1.f / l_sum : 0.f;
-      if constexpr (C::kTmaEpi) {
+      if constexpr (kTmaEpi) {
         // Stage O (bf16) in this row block's Q tile, which no MMA reads any
         // more (its last S MMA completed before the last P*V), in the TMA
         // layout (64-column panels, 128-byte swizzle), then one thread stores
@@ -776,7 +829,9 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           pend_n = (t == 0 && it.T1 == 0) ? 2 : 1;  // row block 1 absent: arrive for it too
         }
       } else {
-        __nv_bfloat16* orow = O + (static_cast<size_t>(it.bh) * N + (row_valid ? q_idx : 0)) * D;
+        __nv_bfloat16* orow =
+            VARLEN ? O + (static_cast<size_t>(it.tok0 + (row_valid ? q_idx : 0)) * Hq + it.bh % Hq) * D
+                   : O + (static_cast<size_t>(it.bh) * N + (row_valid ? q_idx : 0)) * D;
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t r[32];
@@ -799,7 +854,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
     }
     // no store may still be reading shared memory, or writing O, at exit
     release_pending();
-    if (C::kTmaEpi && row == 0) bulk_wait_all();
+    if (kTmaEpi && row == 0) bulk_wait_all();
   }
 
   tc_fence_before();
@@ -839,10 +894,26 @@ bool pp_map(CUtensorMap* m, const void* base, int BH, int rows, int D, int box_r
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int BC, bool CAUSAL>
+// [tokens, H, D] bf16 (variable-length batches), d fastest; box = 64 columns
+// x 1 head x box_rows tokens, so the tile in shared memory is laid out as in
+// pp_map.  Tokens past the end of the tensor read as zeros.
+bool pp_map_thd(CUtensorMap* m, const void* base, int H, int tokens, int D, int box_rows) {
+  auto enc = pp_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(H),
+                        static_cast<cuuint64_t>(tokens)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(H) * D * 2};
+  cuuint32_t box[3] = {64, 1, static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int BC, bool CAUSAL, bool VARLEN>
 int pp_launch(const PrefillLaunch& a) {
   using C = PPCfg<D, BC>;
-  auto kern = prefill_pp_kernel<D, BC, CAUSAL>;
+  auto kern = prefill_pp_kernel<D, BC, CAUSAL, VARLEN>;
   static uint64_t ready = 0;  // one bit per device: attributes set and checked
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return ATTN_ERR_CUDA;
@@ -861,21 +932,36 @@ int pp_launch(const PrefillLaunch& a) {
     ready |= uint64_t(1) << dev;
   }
   CUtensorMap mq, mk, mv, mo;
-  if (!pp_map(&mq, a.Q, a.B * a.Hq, a.N, D, kRows) || !pp_map(&mk, a.K, a.B * a.Hkv, a.N, D, BC) ||
-      !pp_map(&mv, a.V, a.B * a.Hkv, a.N, D, BC) || !pp_map(&mo, a.O, a.B * a.Hq, a.N, D, kRows))
+  if (VARLEN) {
+    if (!pp_map_thd(&mq, a.Q, a.Hq, a.total, D, kRows) ||
+        !pp_map_thd(&mk, a.K, a.Hkv, a.total, D, BC) || !pp_map_thd(&mv, a.V, a.Hkv, a.total, D, BC))
+      return ATTN_ERR_CUDA;
+    mo = mq;  // unused: variable-length batches store O row by row
+    if (a.skip_mask) {  // row blocks past a sequence's end are never visited
+      const size_t n = static_cast<size_t>(a.B) * a.Hq * ((a.N + kRows - 1) / kRows) *
+                       ((a.N + BC - 1) / BC);
+      if (cudaMemsetAsync(a.skip_mask, 2, n, a.stream) != cudaSuccess) return ATTN_ERR_CUDA;
+    }
+  } else if (!pp_map(&mq, a.Q, a.B * a.Hq, a.N, D, kRows) ||
+             !pp_map(&mk, a.K, a.B * a.Hkv, a.N, D, BC) ||
+             !pp_map(&mv, a.V, a.B * a.Hkv, a.N, D, BC) ||
+             !pp_map(&mo, a.O, a.B * a.Hq, a.N, D, kRows)) {
     return ATTN_ERR_CUDA;
+  }
   const long long n_rb = (a.N + kRows - 1) / kRows;
   const long long n_items = static_cast<long long>(a.B) * a.Hq * ((n_rb + 1) / 2);
   const int grid = static_cast<int>(n_items < sm_count[dev] ? n_items : sm_count[dev]);
   kern<<<grid, kPPThreads, C::kSmemBytes, a.stream>>>(
       mq, mk, mv, mo, static_cast<__nv_bfloat16*>(a.O), a.skip_mask, a.status, a.B, a.Hq, a.Hkv, a.N,
-      a.scale_log2, a.tau_log2, a.tau_is_inf, a.wait_limit_ns);
+      a.scale_log2, a.tau_log2, a.tau_is_inf, a.wait_limit_ns, a.cu_seqlens, a.total);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 template <int D, int BC>
 int pp_launch_c(const PrefillLaunch& a) {
-  return a.causal ? pp_launch<D, BC, true>(a) : pp_launch<D, BC, false>(a);
+  if (a.cu_seqlens)
+    return a.causal ? pp_launch<D, BC, true, true>(a) : pp_launch<D, BC, false, true>(a);
+  return a.causal ? pp_launch<D, BC, true, false>(a) : pp_launch<D, BC, false, false>(a);
 }
 
 }  // namespace

@@ -81,6 +81,28 @@ ATTN_API int attn_prefill_ex(const void* Q, const void* K, const void* V, void* 
                     uint8_t* skip_mask);
 
 /*
+ * Prefill over a batch of sequences of different lengths packed one after
+ * another ("varlen"), the layout serving engines batch prompts in:
+ *   Q, O  [total_tokens, Hq, d] and K, V [total_tokens, Hkv, d], bf16, d
+ *         fastest; sequence b is tokens [cu_seqlens[b], cu_seqlens[b+1]).
+ *   cu_seqlens  device int32 [B + 1], non-decreasing, cu_seqlens[B] <=
+ *         total_tokens; lengths above max_seqlen are cut to max_seqlen.  A
+ *         malformed table cannot make the kernel read or write outside the
+ *         tensors (offsets and lengths are clamped to [0, total_tokens]).
+ *   Each sequence attends only to itself (causal: top-left aligned within
+ *   the sequence), with the skip rule of attn_prefill.  Br must be 128
+ *   (Bc 64 or 128).  Rows of O outside every sequence are not written.
+ *   skip_mask (nullable): [B, Hq, ceil(max_seqlen/128), ceil(max_seqlen/Bc)];
+ *   tiles and row blocks past a sequence's end are marked 2.
+ *   Errors: as attn_prefill_ex, plus ATTN_ERR_INVALID_ARG for a null or
+ *   unaligned cu_seqlens, total_tokens or max_seqlen <= 0, or Br != 128.
+ */
+ATTN_API int attn_prefill_varlen(const void* Q, const void* K, const void* V, void* O,
+                                 const int32_t* cu_seqlens, int B, int max_seqlen,
+                                 int total_tokens, int Hq, int Hkv, int d, int causal, float tau,
+                                 int Br, int Bc, void* stream, uint8_t* skip_mask);
+
+/*
  * Prefill with the inputs and the output in host memory: the batch is cut
  * into chunks of `chunk` sequences (0: B/8 rounded up) that flow through two
  * library-owned device buffer sets on two library streams, so the copy of
