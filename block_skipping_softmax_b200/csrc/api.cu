@@ -172,6 +172,43 @@ int attn_prefill_varlen(const void* Q, const void* K, const void* V, void* O,
   return bss::launch_prefill_pp(a);
 }
 
+int attn_prefill_qk8(const void* Q8, const void* K8, const float* q_scales, const float* k_scales,
+                     const void* V, void* O, int B, int Hq, int Hkv, int N, int d, int causal,
+                     float tau, int Br, int Bc, void* stream, uint8_t* skip_mask) {
+  if (!q_scales || !k_scales) return ATTN_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(q_scales) & 3u) || (reinterpret_cast<uintptr_t>(k_scales) & 3u))
+    return ATTN_ERR_INVALID_ARG;
+  if (d != 128 || Br != 128) return ATTN_ERR_INVALID_ARG;
+  int st = check_prefill(Q8, K8, V, O, B, Hq, Hkv, N, d, tau, Br, Bc);
+  if (st != ATTN_OK) return st;
+  int dev = 0;
+  int* status = nullptr;
+  if ((st = device_ready(&dev, &status)) != ATTN_OK) return st;
+  bss::PrefillLaunch a{};
+  a.Q = Q8;
+  a.K = K8;
+  a.V = V;
+  a.O = O;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.N = N;
+  a.d = d;
+  a.causal = causal ? 1 : 0;
+  a.Br = Br;
+  a.Bc = Bc;
+  a.scale_log2 = kLog2e / std::sqrt(static_cast<float>(d));
+  a.tau_is_inf = std::isinf(tau) ? 1 : 0;
+  a.tau_log2 = a.tau_is_inf ? 0.f : tau * kLog2e;
+  a.skip_mask = skip_mask;
+  a.status = status;
+  a.wait_limit_ns = g_wait_limit_ns;
+  a.stream = static_cast<cudaStream_t>(stream);
+  a.q_scales = q_scales;
+  a.k_scales = k_scales;
+  return bss::launch_prefill_pp(a);
+}
+
 int attn_prefill(const void* Q, const void* K, const void* V, void* O, int B, int Hq, int Hkv,
                  int N, int d, int causal, float tau, int Br, int Bc) {
   return attn_prefill_ex(Q, K, V, O, B, Hq, Hkv, N, d, causal, tau, Br, Bc, g_stream, nullptr);

@@ -28,6 +28,11 @@ struct PrefillLaunch {
   // and N is the longest sequence
   const int* cu_seqlens;
   int total;
+  // e4m3 Q and K (q_scales != nullptr): Q [B, Hq, N, d] and K [B, Hkv, N, d]
+  // hold one byte per element, head slab (b, h) scaled by q_scales[b*Hq+h]
+  // (k_scales[b*Hkv+h]); V and O stay bf16
+  const float* q_scales;
+  const float* k_scales;
 };
 
 int launch_prefill(const PrefillLaunch& a);     // one row block per CTA (any Br)

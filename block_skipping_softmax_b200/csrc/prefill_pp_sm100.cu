@@ -58,28 +58,36 @@ constexpr float kRescale = 8.0f;  // lazy rescale threshold (log2 units)
 #endif
 constexpr uint32_t kPolyPairs = BSS_POLY_PAIRS;
 
-template <int D, int BC>
+// QK8: Q and K arrive as e4m3 (one byte per element, 128-byte rows hold 128
+// columns) and S = Q K^T runs as kind::f8f6f4 MMAs; V and P stay bf16.
+template <int D, int BC, bool QK8 = false>
 struct PPCfg {
-  static constexpr int kPanels = D / 64;
-  static constexpr int kQTile = kRows * D * 2;
+  static constexpr int kEB = QK8 ? 1 : 2;                 // bytes per Q/K element
+  static constexpr int kQKPanels = D * kEB / 128;        // 128-byte column panels of Q and K
+  static constexpr int kVPanels = D / 64;                // of V (bf16)
+  static constexpr int kQKCols = 128 / kEB;              // Q/K columns per panel
+  static constexpr int kSSteps = D * kEB / 32;           // S MMAs per tile (32 bytes of K each)
+  static constexpr int kQTile = kRows * D * kEB;
   static constexpr int kQPanel = kRows * 128;
-  static constexpr int kKVBytes = BC * D * 2;
+  static constexpr int kKBytes = BC * D * kEB;
+  static constexpr int kVBytes = BC * D * 2;
   static constexpr int kKVPanel = BC * 128;
-  static constexpr int kKS = (BC == 128 && D == 128) ? 2 : 3;
-  static constexpr int kVS = (BC == 128 && D == 128) ? 2 : 3;
+  static constexpr int kKS = (BC == 128 && D == 128 && !QK8) ? 2 : 3;
+  static constexpr int kVS = (BC == 128 && D == 128 && !QK8) ? 2 : 3;
   // S/P buffers per row block: two when TMEM has room (Bc = 64), so the MMA
   // for key tile j+1 runs while the softmax works on tile j
   static constexpr int kSB = (2 * D + 4 * BC <= 512) ? 2 : 1;
   // Q slots: with two, the next work item's Q loads while this one runs
-  static constexpr int kQS = (BC == 128 && D == 128) ? 1 : 2;
+  static constexpr int kQS = (BC == 128 && D == 128 && !QK8) ? 1 : 2;
   static constexpr int kQSlot = 2 * kQTile;  // two row blocks
   // With two Q slots, a row block's O is staged in its own (finished) Q tile
-  // and written by a TMA store; the slot is released once the store has read it.
-  static constexpr bool kTmaEpi = kQS == 2;
+  // and written by a TMA store; the slot is released once the store has read
+  // it.  An e4m3 Q tile is too small to hold the bf16 O tile.
+  static constexpr bool kTmaEpi = kQS == 2 && !QK8;
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQS * kQSlot;
-  static constexpr int kOffV = kOffK + kKS * kKVBytes;
-  static constexpr int kOffBar = kOffV + kVS * kKVBytes;
+  static constexpr int kOffV = kOffK + kKS * kKBytes;
+  static constexpr int kOffBar = kOffV + kVS * kVBytes;
   // k_full[KS], v_full[VS], commit ring[2][CR], p_full[2][SB], dec[2][DR],
   // q_full[QS], q_empty[QS], mma_done
   static constexpr int kNumBars = kKS + kVS + 2 * kCR + 2 * kSB + 2 * kDR + 2 * kQS + 1;
@@ -208,7 +216,7 @@ struct Pending3 {
 
 }  // namespace
 
-template <int D, int BC, bool CAUSAL, bool VARLEN>
+template <int D, int BC, bool CAUSAL, bool VARLEN, bool QK8>
 __global__ void __launch_bounds__(kPPThreads, 1)
     prefill_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -216,8 +224,9 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                       uint8_t* __restrict__ skip_mask, int* __restrict__ status, int B, int Hq,
                       int Hkv, int N, float scale_log2, float tau_log2, int tau_is_inf,
                       unsigned long long wait_limit_ns, const int* __restrict__ cu_seqlens,
-                      int total) {
-  using C = PPCfg<D, BC>;
+                      int total, const float* __restrict__ q_scales,
+                      const float* __restrict__ k_scales) {
+  using C = PPCfg<D, BC, QK8>;
   // variable-length batches store O row by row: a TMA store of the last row
   // block would write into the next sequence's rows
   constexpr bool kTmaEpi = C::kTmaEpi && !VARLEN;
@@ -328,13 +337,13 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         const int nq = it.T1 > 0 ? 2 : 1;
         mbar_arrive_expect_tx(b_q_full(qs), nq * C::kQTile);
         for (int t = 0; t < nq; ++t)
-          for (int p = 0; p < C::kPanels; ++p)
+          for (int p = 0; p < C::kQKPanels; ++p)
             if constexpr (VARLEN)  // Q as [tokens, Hq, d]
               tma_load_3d(sQ + qs * C::kQSlot + t * C::kQTile + p * C::kQPanel, &tmQ, b_q_full(qs),
-                          p * 64, it.bh % Hq, it.tok0 + (it.rb0 + t) * kRows);
+                          p * C::kQKCols, it.bh % Hq, it.tok0 + (it.rb0 + t) * kRows);
             else
               tma_load_3d(sQ + qs * C::kQSlot + t * C::kQTile + p * C::kQPanel, &tmQ, b_q_full(qs),
-                          p * 64, (it.rb0 + t) * kRows, it.bh);
+                          p * C::kQKCols, (it.rb0 + t) * kRows, it.bh);
         for (int j = 0; j < it.Tmax; ++j) {
           const int s = kload % C::kKS;
           if (pend.n == C::kKS) {  // the slot's previous tile: its S MMAs must have run
@@ -345,14 +354,14 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             }
             pend.pop();
           }
-          mbar_arrive_expect_tx(b_k_full(s), C::kKVBytes);
-          for (int p = 0; p < C::kPanels; ++p) {
+          mbar_arrive_expect_tx(b_k_full(s), C::kKBytes);
+          for (int p = 0; p < C::kQKPanels; ++p) {
             if constexpr (VARLEN)  // K as [tokens, Hkv, d]
-              tma_load_3d(sK + s * C::kKVBytes + p * C::kKVPanel, &tmK, b_k_full(s), p * 64,
+              tma_load_3d(sK + s * C::kKBytes + p * C::kKVPanel, &tmK, b_k_full(s), p * C::kQKCols,
                           (it.bh % Hq) / g, it.tok0 + j * BC);
             else
-              tma_load_3d(sK + s * C::kKVBytes + p * C::kKVPanel, &tmK, b_k_full(s), p * 64, j * BC,
-                          bkv);
+              tma_load_3d(sK + s * C::kKBytes + p * C::kKVPanel, &tmK, b_k_full(s), p * C::kQKCols,
+                          j * BC, bkv);
           }
           // K tile j is read by S of row block 1 last (if it exists, T1 >= T0)
           if (j < it.T1) pend.push(1, base1 + j, 0);
@@ -396,13 +405,13 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             pend.pop();
           }
           const int s = vload % C::kVS;
-          mbar_arrive_expect_tx(b_v_full(s), C::kKVBytes);
-          for (int p = 0; p < C::kPanels; ++p) {
+          mbar_arrive_expect_tx(b_v_full(s), C::kVBytes);
+          for (int p = 0; p < C::kVPanels; ++p) {
             if constexpr (VARLEN)  // V as [tokens, Hkv, d]
-              tma_load_3d(sV + s * C::kKVBytes + p * C::kKVPanel, &tmV, b_v_full(s), p * 64,
+              tma_load_3d(sV + s * C::kVBytes + p * C::kKVPanel, &tmV, b_v_full(s), p * 64,
                           (it.bh % Hq) / g, it.tok0 + j * BC);
             else
-              tma_load_3d(sV + s * C::kKVBytes + p * C::kKVPanel, &tmV, b_v_full(s), p * 64, j * BC,
+              tma_load_3d(sV + s * C::kVBytes + p * C::kKVPanel, &tmV, b_v_full(s), p * 64, j * BC,
                           bkv);
           }
           // P*V of tile j, row block 1 (if it visits j) is issued after row block 0's
@@ -450,7 +459,8 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         mbar_drain(b_v_full(t % C::kVS), (t / C::kVS) & 1, wait_limit_ns);
     } else if (warp == 1 && lane == 0) {
       // ---------------------------------------------------- MMA issuer
-      constexpr uint32_t idS = idesc_bf16_f32(kRows, BC, false, false);
+      constexpr uint32_t idS =
+          QK8 ? idesc_e4m3_f32(kRows, BC) : idesc_bf16_f32(kRows, BC, false, false);
       constexpr uint32_t idPV = idesc_bf16_f32(kRows, D, false, true);
       int kuse = 0, vuse = 0, items = 0;
       int pc[2] = {0, 0}, dc[2] = {0, 0}, sq[2] = {0, 0}, cmc[2] = {0, 0};
@@ -463,13 +473,17 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       uint32_t dQ = sw128_desc_lo(sQ, 16);  // this item's Q slot
       auto issue_S = [&](int t, int kslot, int buf) {
         const uint32_t a0 = dQ + t * (C::kQTile >> 4);
-        const uint32_t b0 = dK0 + kslot * (C::kKVBytes >> 4);
+        const uint32_t b0 = dK0 + kslot * (C::kKBytes >> 4);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < C::kSSteps; ++kk) {  // 32 bytes of the reduction each
           const uint32_t oq = ((kk >> 2) * C::kQPanel + (kk & 3) * 32) >> 4;
           const uint32_t ok_ = ((kk >> 2) * C::kKVPanel + (kk & 3) * 32) >> 4;
-          mma_ss(tS(t, buf), desc_join(a0 + oq, kHi), desc_join(b0 + ok_, kHi), idS,
-                 kk > 0 ? 1u : 0u);
+          if constexpr (QK8)
+            mma_ss_f8(tS(t, buf), desc_join(a0 + oq, kHi), desc_join(b0 + ok_, kHi), idS,
+                      kk > 0 ? 1u : 0u);
+          else
+            mma_ss(tS(t, buf), desc_join(a0 + oq, kHi), desc_join(b0 + ok_, kHi), idS,
+                   kk > 0 ? 1u : 0u);
         }
       };
       auto commit = [&](int t) {
@@ -534,7 +548,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                 tc_fence_after();
                 v_used = true;
               }
-              const uint32_t vb = dV0 + (vuse % C::kVS) * (C::kKVBytes >> 4);
+              const uint32_t vb = dV0 + (vuse % C::kVS) * (C::kVBytes >> 4);
 #pragma unroll
               for (int kk = 0; kk < BC / 16; ++kk)
                 mma_ts(tO(t), tS(t, pb) + kk * 8, desc_join(vb + ((kk * 16 * 128) >> 4), kHi), idPV,
@@ -608,6 +622,11 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       const size_t mask_base =
           skip_mask ? ((static_cast<size_t>(it.bh) * n_rb + rb) * n_tiles) : 0;
       float m_exact = NEG_INF, m_ref = NEG_INF, l_sum = 0.f;
+      // log2-domain score scale; e4m3 scores carry the two per-head scales
+      float sl2 = scale_log2;
+      if constexpr (QK8)
+        sl2 *= __ldg(q_scales + it.bh) *
+               __ldg(k_scales + (it.bh / Hq) * Hkv + (it.bh % Hq) / (Hq / Hkv));
       for (int j = 0; j < T; ++j) {
         const int sb = sc % SB;  // S/P buffer of key tile j
         ++sc;
@@ -637,7 +656,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
 #pragma unroll
             for (int k = 0; k < 4; ++k)
               m4[k] = fmax3(m4[k], __uint_as_float(u[c + 2 * k]), __uint_as_float(u[c + 2 * k + 1]));
-          mt = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * scale_log2;  // log2 units; -inf stays -inf
+          mt = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * sl2;  // log2 units; -inf stays -inf
         }
         // ---- skip test: every row of this row block must have mt < m - tau.
         // Each warp publishes its own verdict (all its rows pass, or not) and
@@ -711,7 +730,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         // pack to bf16 for the P*V MMA; the row sum adds the fp32 pair with
         // one packed add (four independent chains)
         const float neg_m = row_valid ? -m_ref : 0.f;  // invalid rows: all scores -inf -> P = 0
-        const float2 sc2 = make_float2(scale_log2, scale_log2);
+        const float2 sc2 = make_float2(sl2, sl2);
         const float2 nm2 = make_float2(neg_m, neg_m);
         float2 rs2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                          make_float2(0.f, 0.f)};  // four independent add chains
@@ -822,7 +841,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         if (row == 0) {
           release_pending();  // at most one store in flight per warpgroup
 #pragma unroll
-          for (int p = 0; p < C::kPanels; ++p)
+          for (int p = 0; p < C::kVPanels; ++p)
             tma_store_3d(&tmO, stage + p * C::kQPanel, p * 64, rb * kRows, it.bh);
           bulk_commit_group();
           pend_slot = qs;
@@ -894,6 +913,21 @@ bool pp_map(CUtensorMap* m, const void* base, int BH, int rows, int D, int box_r
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [BH, N, D] e4m3 (one byte per element), d fastest; box = 128 columns (one
+// 128-byte swizzle row) x box_rows rows.
+bool pp_map_e4m3(CUtensorMap* m, const void* base, int BH, int N, int D, int box_rows) {
+  auto enc = pp_encoder();
+  if (!enc) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N),
+                        static_cast<cuuint64_t>(BH)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(N) * D};
+  cuuint32_t box[3] = {128, static_cast<cuuint32_t>(box_rows), 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // [tokens, H, D] bf16 (variable-length batches), d fastest; box = 64 columns
 // x 1 head x box_rows tokens, so the tile in shared memory is laid out as in
 // pp_map.  Tokens past the end of the tensor read as zeros.
@@ -910,10 +944,10 @@ bool pp_map_thd(CUtensorMap* m, const void* base, int H, int tokens, int D, int 
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int BC, bool CAUSAL, bool VARLEN>
+template <int D, int BC, bool CAUSAL, bool VARLEN, bool QK8>
 int pp_launch(const PrefillLaunch& a) {
-  using C = PPCfg<D, BC>;
-  auto kern = prefill_pp_kernel<D, BC, CAUSAL, VARLEN>;
+  using C = PPCfg<D, BC, QK8>;
+  auto kern = prefill_pp_kernel<D, BC, CAUSAL, VARLEN, QK8>;
   static uint64_t ready = 0;  // one bit per device: attributes set and checked
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return ATTN_ERR_CUDA;
@@ -942,6 +976,12 @@ int pp_launch(const PrefillLaunch& a) {
                        ((a.N + BC - 1) / BC);
       if (cudaMemsetAsync(a.skip_mask, 2, n, a.stream) != cudaSuccess) return ATTN_ERR_CUDA;
     }
+  } else if (QK8) {
+    if (!pp_map_e4m3(&mq, a.Q, a.B * a.Hq, a.N, D, kRows) ||
+        !pp_map_e4m3(&mk, a.K, a.B * a.Hkv, a.N, D, BC) ||
+        !pp_map(&mv, a.V, a.B * a.Hkv, a.N, D, BC))
+      return ATTN_ERR_CUDA;
+    mo = mv;  // unused: e4m3 Q tiles cannot stage O, which is stored row by row
   } else if (!pp_map(&mq, a.Q, a.B * a.Hq, a.N, D, kRows) ||
              !pp_map(&mk, a.K, a.B * a.Hkv, a.N, D, BC) ||
              !pp_map(&mv, a.V, a.B * a.Hkv, a.N, D, BC) ||
@@ -953,21 +993,30 @@ int pp_launch(const PrefillLaunch& a) {
   const int grid = static_cast<int>(n_items < sm_count[dev] ? n_items : sm_count[dev]);
   kern<<<grid, kPPThreads, C::kSmemBytes, a.stream>>>(
       mq, mk, mv, mo, static_cast<__nv_bfloat16*>(a.O), a.skip_mask, a.status, a.B, a.Hq, a.Hkv, a.N,
-      a.scale_log2, a.tau_log2, a.tau_is_inf, a.wait_limit_ns, a.cu_seqlens, a.total);
+      a.scale_log2, a.tau_log2, a.tau_is_inf, a.wait_limit_ns, a.cu_seqlens, a.total, a.q_scales,
+      a.k_scales);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
 template <int D, int BC>
 int pp_launch_c(const PrefillLaunch& a) {
   if (a.cu_seqlens)
-    return a.causal ? pp_launch<D, BC, true, true>(a) : pp_launch<D, BC, false, true>(a);
-  return a.causal ? pp_launch<D, BC, true, false>(a) : pp_launch<D, BC, false, false>(a);
+    return a.causal ? pp_launch<D, BC, true, true, false>(a) : pp_launch<D, BC, false, true, false>(a);
+  return a.causal ? pp_launch<D, BC, true, false, false>(a) : pp_launch<D, BC, false, false, false>(a);
 }
 
 }  // namespace
 
 int launch_prefill_pp(const PrefillLaunch& a) {
   if (a.Br != 128) return ATTN_ERR_INVALID_ARG;
+  if (a.q_scales) {  // e4m3 Q and K: d = 128, fixed-length batches
+    if (a.d != 128 || a.cu_seqlens) return ATTN_ERR_INVALID_ARG;
+    if (a.Bc == 64)
+      return a.causal ? pp_launch<128, 64, true, false, true>(a)
+                      : pp_launch<128, 64, false, false, true>(a);
+    return a.causal ? pp_launch<128, 128, true, false, true>(a)
+                    : pp_launch<128, 128, false, false, true>(a);
+  }
   if (a.d == 128) return a.Bc == 64 ? pp_launch_c<128, 64>(a) : pp_launch_c<128, 128>(a);
   if (a.d == 64) return a.Bc == 64 ? pp_launch_c<64, 64>(a) : pp_launch_c<64, 128>(a);
   return ATTN_ERR_INVALID_ARG;

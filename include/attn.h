@@ -103,6 +103,41 @@ ATTN_API int attn_prefill_varlen(const void* Q, const void* K, const void* V, vo
                                  int Br, int Bc, void* stream, uint8_t* skip_mask);
 
 /*
+ * e4m3 quantisation (for attn_prefill_qk8).  x is a device tensor of
+ * groups * group_elems bf16 values, cut into `groups` contiguous groups
+ * (one head slab [N, d] each for Q [B, Hq, N, d] or K [B, Hkv, N, d]).
+ * Group g gets the scale s = 2^k, k the smallest integer >= -126 with
+ * max|x| <= 448 * 2^k (448: the largest finite e4m3 value); a group of zeros
+ * gets 1, a group holding inf or NaN gets NaN.  q[i] = e4m3(x[i] / s), rounded
+ * to nearest, ties to even (OCP FP8 E4M3: bias 7, no infinities).  Since s is
+ * a power of two, q * s is exactly representable in bf16.
+ *   x: const bf16*, 16-byte aligned.  q: uint8_t* of the same element count,
+ *   16-byte aligned.  scales: float* [groups], 4-byte aligned.  All device
+ *   memory owned by the caller; the call is asynchronous on `stream`.
+ *   Errors: ATTN_ERR_INVALID_ARG for null or unaligned pointers, groups or
+ *   group_elems <= 0, or group_elems not a multiple of 16;
+ *   ATTN_ERR_UNSUPPORTED off sm_100 or beyond 2^31 blocks; ATTN_ERR_CUDA.
+ */
+ATTN_API int attn_quantize_e4m3(const void* x, void* q, float* scales, long long groups,
+                                long long group_elems, void* stream);
+
+/*
+ * Prefill with S = Q K^T from e4m3 operands on the FP8 tensor cores (kind
+ * f8f6f4, fp32 accumulation); P*V stays bf16.  Q8 [B, Hq, N, d] and K8
+ * [B, Hkv, N, d] hold one byte per element as written by attn_quantize_e4m3
+ * with one group per head slab; head (b, h) of Q means Q8 * q_scales[b*Hq+h]
+ * and head (b, h) of K means K8 * k_scales[b*Hkv+h].  The result is attention
+ * (with the skip rule of attn_prefill) over those dequantised Q and K.
+ * V, O and skip_mask as attn_prefill_ex.  d = 128 and Br = 128 only.
+ *   Errors: as attn_prefill_ex, plus ATTN_ERR_INVALID_ARG for null or
+ *   unaligned scale pointers, d != 128 or Br != 128.
+ */
+ATTN_API int attn_prefill_qk8(const void* Q8, const void* K8, const float* q_scales,
+                              const float* k_scales, const void* V, void* O, int B, int Hq,
+                              int Hkv, int N, int d, int causal, float tau, int Br, int Bc,
+                              void* stream, uint8_t* skip_mask);
+
+/*
  * Prefill with the inputs and the output in host memory: the batch is cut
  * into chunks of `chunk` sequences (0: B/8 rounded up) that flow through two
  * library-owned device buffer sets on two library streams, so the copy of

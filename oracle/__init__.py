@@ -66,6 +66,10 @@ def _load(path: str | None = None):
     lib.oracle_decode.restype = ci
     lib.oracle_decode.argtypes = [u16p, u16p, u16p, ci, ci, ci, ci, ci, ctypes.c_double, ci, ci,
                                   ci, f64p, f64p, u8p, f64p, f64p, ci]
+    lib.oracle_e4m3_value.restype = ctypes.c_double
+    lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+    lib.oracle_quantize_e4m3.restype = ci
+    lib.oracle_quantize_e4m3.argtypes = [u16p, ctypes.c_int64, ctypes.c_int64, u8p, f64p]
     if path is None:
         _lib = lib
     return lib
@@ -161,3 +165,31 @@ def decode(q, K, V, tau: float, Ls: int, Bt: int = 64, want_exact: bool = True,
 
 
 INF = math.inf
+
+
+def e4m3_values(lib_path: str | None = None) -> np.ndarray:
+    """fp64 value of each of the 256 e4m3 codes (NaN for the two NaN codes)."""
+    lib = _load(lib_path)
+    return np.array([lib.oracle_e4m3_value(c) for c in range(256)])
+
+
+def quantize_e4m3(x, groups: int, lib_path: str | None = None):
+    """e4m3 codes (uint8, x's shape) and fp64 power-of-two scales [groups] of a
+    bf16 tensor cut into ``groups`` equal contiguous groups."""
+    xb = _bits(x)
+    n = xb.size
+    if groups <= 0 or n % groups:
+        raise ValueError("quantize_e4m3: the element count must split into equal groups")
+    codes = np.empty(xb.shape, dtype=np.uint8)
+    scales = np.empty(groups)
+    st = _load(lib_path).oracle_quantize_e4m3(_p(xb, ctypes.c_uint16), groups, n // groups,
+                                              _p(codes, ctypes.c_uint8), _p(scales, ctypes.c_double))
+    if st != 0:
+        raise ValueError(f"oracle_quantize_e4m3 failed with status {st}")
+    return codes, scales
+
+
+def dequantize_e4m3(codes: np.ndarray, scales: np.ndarray, lib_path: str | None = None) -> np.ndarray:
+    """fp64 values code * scale, one scale per equal contiguous group."""
+    vals = e4m3_values(lib_path)[codes.reshape(scales.size, -1)]
+    return (vals * scales[:, None]).reshape(codes.shape)

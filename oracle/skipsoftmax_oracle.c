@@ -429,3 +429,89 @@ int oracle_decode(const uint16_t *q, const uint16_t *K, const uint16_t *V,
     }
     return status;
 }
+
+/*
+ * e4m3 quantisation for the FP8 Q K^T path (the page names FP8 attention as
+ * the path the skip rule combines with; the scale rule is this library's
+ * own, stated here in full).
+ *
+ * Format (OCP 8-bit floating point, E4M3): sign bit, 4 exponent bits with
+ * bias 7, 3 mantissa bits; exponent field 0 holds the subnormals
+ * m * 2^-9 (m = 0..7); field 15 with mantissa 7 is NaN; there are no
+ * infinities, and the largest finite value is 1.75 * 2^8 = 448.
+ *
+ * Quantisation of one group x[0..n): s = 2^k with k the smallest integer
+ * >= -126 such that max|x| <= 448 * 2^k (s = 1 for a group of zeros, NaN for
+ * a group holding inf or NaN); code_i = the e4m3 value nearest to x_i / s,
+ * ties to the code with an even mantissa.
+ */
+double oracle_e4m3_value(uint8_t code)
+{
+    const int sign = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    double v;
+    if (e == 15 && m == 7)
+        return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);
+    else
+        v = ldexp(1.0 + m / 8.0, e - 7);
+    return sign ? -v : v;
+}
+
+/* Nearest code to y (|y| <= 448), ties to even: the non-negative codes
+ * 0..126 are in increasing order of value, so find (by bisection) the last
+ * code whose value does not exceed |y| and compare it with the next one. */
+static uint8_t e4m3_nearest(double y)
+{
+    const double a = fabs(y);
+    int lo = 0, hi = 126;  /* value(lo) <= a always; the answer lies in [lo, hi] */
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) / 2;
+        if (oracle_e4m3_value((uint8_t)mid) <= a)
+            lo = mid;
+        else
+            hi = mid - 1;
+    }
+    int c = lo;
+    if (lo < 126) {
+        const double dl = a - oracle_e4m3_value((uint8_t)lo);
+        const double dh = oracle_e4m3_value((uint8_t)(lo + 1)) - a;
+        if (dh < dl || (dh == dl && ((lo + 1) & 1) == 0))
+            c = lo + 1;
+    }
+    return (uint8_t)(c | ((y < 0 || (y == 0 && signbit(y))) ? 0x80 : 0));
+}
+
+int oracle_quantize_e4m3(const uint16_t *x, int64_t groups, int64_t group_elems, uint8_t *q,
+                         double *scales)
+{
+    if (!x || !q || !scales || groups <= 0 || group_elems <= 0)
+        return ORACLE_BAD_ARG;
+    for (int64_t g = 0; g < groups; ++g) {
+        const uint16_t *xg = x + g * group_elems;
+        double amax = 0.0;
+        int finite = 1;
+        for (int64_t i = 0; i < group_elems; ++i) {
+            const double v = widen_bf16(xg[i]);
+            if (!isfinite(v))
+                finite = 0;
+            else if (fabs(v) > amax)
+                amax = fabs(v);
+        }
+        double s;
+        if (!finite) {
+            s = NAN;
+        } else if (amax == 0.0) {
+            s = 1.0;
+        } else {
+            int k = -126;
+            while (amax > ldexp(448.0, k))
+                ++k;
+            s = ldexp(1.0, k);
+        }
+        scales[g] = s;
+        for (int64_t i = 0; i < group_elems; ++i)
+            q[g * group_elems + i] = finite ? e4m3_nearest(widen_bf16(xg[i]) / s) : 0x7f;
+    }
+    return ORACLE_OK;
+}

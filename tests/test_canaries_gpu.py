@@ -64,6 +64,42 @@ def test_prefill_writes_only_its_outputs(Br, Bc, causal, tau):
     assert torch.equal(gm.inner.view(B, Hq, n_rb, n_t), ref_m)
 
 
+@pytest.mark.parametrize("Bc", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_prefill_qk8_writes_only_its_outputs(Bc, causal):
+    B, Hq, Hkv, N, d = 2, 4, 2, 333, 128
+    Q, K, V = inputs.prefill_inputs(B, Hq, Hkv, N, d, seed=53, q_sigma=2.0, q_u=8.0, sink_scale=6.0)
+    Q8, qs = bss.quantize_e4m3(Q.cuda())
+    K8, ks = bss.quantize_e4m3(K.cuda())
+    Vd = V.cuda()
+    ref_o, ref_m = bss.prefill_qk8(Q8, K8, qs, ks, Vd, causal, 2.0, 128, Bc, skip_mask=True)
+    n_rb, n_t = -(-N // 128), -(-N // Bc)
+    go = Guarded(B * Hq * N * d * 2)
+    gm = Guarded(B * Hq * n_rb * n_t)
+    st = bss.attn_prefill_qk8(Q8.data_ptr(), K8.data_ptr(), qs.data_ptr(), ks.data_ptr(), Vd.data_ptr(),
+                              go.ptr(), B, Hq, Hkv, N, d, causal, 2.0, 128, Bc,
+                              torch.cuda.current_stream().cuda_stream, gm.ptr())
+    assert st == 0
+    assert bss.attn_sync_status() == 0
+    assert go.intact() and gm.intact()
+    assert torch.equal(go.inner.view(torch.bfloat16).view(B, Hq, N, d), ref_o)
+    assert torch.equal(gm.inner.view(B, Hq, n_rb, n_t), ref_m)
+
+
+def test_quantize_writes_only_its_outputs():
+    x = torch.randn(2, 3, 333, 128, dtype=torch.float32).to(torch.bfloat16).cuda()
+    ref_q, ref_s = bss.quantize_e4m3(x)
+    gq = Guarded(x.numel())
+    gs = Guarded(2 * 3 * 4)
+    st = bss.attn_quantize_e4m3(x.data_ptr(), gq.ptr(), gs.ptr(), 6, 333 * 128,
+                                torch.cuda.current_stream().cuda_stream)
+    assert st == 0
+    torch.cuda.synchronize()
+    assert gq.intact() and gs.intact()
+    assert torch.equal(gq.inner.view(2, 3, 333, 128), ref_q)
+    assert torch.equal(gs.inner.view(torch.float32).view(2, 3), ref_s)
+
+
 @pytest.mark.parametrize("rule", [0, 1, 2, 3])
 def test_decode_writes_only_its_outputs(rule):
     B, Hq, Hkv, L, d = 3, 8, 2, 1999, 128

@@ -30,6 +30,11 @@ MUTANTS = {
     "per_head_uses_group_margin": (
         "if (per_head && row_margin(mt[r], m[r], tau) < 0.0) {",
         "if (per_head && margin_j < 0.0) {"),
+    "e4m3_ties_to_odd": ("((lo + 1) & 1) == 0)", "((lo + 1) & 1) == 1)"),
+    "e4m3_ties_away_from_zero": ("(dh == dl && ((lo + 1) & 1) == 0)", "(dh == dl)"),
+    "e4m3_subnormal_exponent": ("v = ldexp((double)m, -9);", "v = ldexp((double)m, -10);"),
+    "e4m3_scale_not_smallest": ("while (amax > ldexp(448.0, k))", "while (amax >= ldexp(448.0, k))"),
+    "e4m3_sign_dropped": ("? 0x80 : 0));", "? 0x00 : 0));"),
     "sink_seed_from_second_tile": (
         "for (int c = 0; c < Bt && c < L; ++c)", "for (int c = Bt; c < 2 * Bt && c < L; ++c)"),
 }

@@ -480,6 +480,87 @@ def pin_decode_rule_variants_from_definition(lib):
         np.testing.assert_allclose(a["o"], b_["o"], rtol=0, atol=1e-13)
 
 
+# ----------------------------------------------------------------------------
+# e4m3 quantisation (FP8 Q K^T path)
+# ----------------------------------------------------------------------------
+
+def bf16_bits(vals):
+    t = torch.tensor(np.asarray(vals, np.float64)).to(torch.bfloat16)
+    assert np.array_equal(t.double().numpy(), np.asarray(vals, np.float64)), "value not exact in bf16"
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+@pin
+def pin_e4m3_code_values(lib):
+    """The 256 code values equal the library's float8_e4m3fn decoding and the
+    format's fixed points: 448 the largest, 2^-9 the smallest subnormal,
+    2^-6 the smallest normal, 1 and -1, the two NaNs."""
+    v = oracle.e4m3_values(lib_path=lib)
+    ref = torch.arange(256, dtype=torch.uint8).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    np.testing.assert_array_equal(v, ref)
+    assert v[0x7E] == 448.0 and v[0x01] == 2.0 ** -9 and v[0x08] == 2.0 ** -6
+    assert v[0x38] == 1.0 and v[0xB8] == -1.0 and v[0x80] == 0.0 and np.signbit(v[0x80])
+    assert np.isnan(v[0x7F]) and np.isnan(v[0xFF]) and np.isfinite(np.delete(v, [0x7F, 0xFF])).all()
+
+
+@pin
+def pin_e4m3_rounding_and_ties(lib):
+    """Codes are round-to-nearest, ties to the even mantissa, with the sign
+    kept: midpoints between neighbours (normal and subnormal) go to the even
+    code; random data equals the library's RNE cast of x / s."""
+    # one group with max 448 (scale 1): exact midpoints and their images
+    mids = [448.0, 1.0625, 1.1875, 2.0 ** -10, 3 * 2.0 ** -10, -1.0625, -(2.0 ** -10), 432.0, 13 * 2.0 ** -10]
+    want = [0x7E, 0x38, 0x3A, 0x00, 0x02, 0xB8, 0x80, 0x7E, 0x06]
+    codes, scales = oracle.quantize_e4m3(bf16_bits(mids), 1, lib_path=lib)
+    assert scales[0] == 1.0
+    assert list(codes) == want, [hex(c) for c in codes]
+    g = torch.Generator().manual_seed(3)
+    x = (torch.randn(12, 2048, generator=g, dtype=torch.float64)
+         * torch.logspace(-6, 6, 12, base=2.0, dtype=torch.float64)[:, None]).to(torch.bfloat16)
+    x[3, :100] = 0.0
+    x[4, 7] = -0.0
+    codes, scales = oracle.quantize_e4m3(x, 12, lib_path=lib)
+    cast = (x.double() / torch.tensor(scales)[:, None]).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(codes, cast)
+    deq = oracle.dequantize_e4m3(codes, scales, lib_path=lib)
+    v = oracle.e4m3_values(lib_path=lib)
+    step = np.diff(v[:127])  # spacing above each non-negative code
+    for r in range(12):  # |error| <= half the local spacing
+        a = np.abs(x[r].double().numpy()) / scales[r]
+        c = np.searchsorted(v[:127], a, side="right") - 1
+        half = step[np.minimum(c, 125)] / 2
+        assert np.all(np.abs(deq[r] - x[r].double().numpy()) <= half * scales[r] + 0.0)
+
+
+@pin
+def pin_e4m3_scale_rule(lib):
+    """Scale = smallest power of two 2^k (k >= -126) with max|x| <= 448 * 2^k:
+    exact boundaries, one bf16 step above them, zeros, tiny and non-finite
+    groups; the largest code of a normal group lies in (224, 448]."""
+    for k in (-20, -3, 0, 1, 7, 40):
+        at = 448.0 * 2.0 ** k
+        above = float(torch.tensor(at, dtype=torch.bfloat16).view(torch.int16).add(1).view(torch.bfloat16))
+        c, s = oracle.quantize_e4m3(bf16_bits([at, -1.0 * 2.0 ** k, 0.0, 0.0]), 1, lib_path=lib)
+        assert s[0] == 2.0 ** k and c[0] == 0x7E
+        c, s = oracle.quantize_e4m3(bf16_bits([0.5 * 2.0 ** k, -above, 0.0, 0.0]), 1, lib_path=lib)
+        assert above == 450.0 * 2.0 ** k
+        assert s[0] == 2.0 ** (k + 1) and c[1] == 0xF6  # -225 rounds to -224 = -1.75 * 2^7 (code 0xF6)
+    _, s = oracle.quantize_e4m3(bf16_bits([0.0] * 16), 2, lib_path=lib)
+    assert list(s) == [1.0, 1.0]
+    _, s = oracle.quantize_e4m3(bf16_bits([2.0 ** -130, 0.0, 0.0, 0.0]), 1, lib_path=lib)
+    assert s[0] == 2.0 ** -126
+    inf16 = torch.tensor([1.0, float("inf"), 2.0, 3.0], dtype=torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    _, s = oracle.quantize_e4m3(inf16, 2, lib_path=lib)
+    assert np.isnan(s[0]) and s[1] == 2.0 ** -7
+    g = torch.Generator().manual_seed(5)
+    x = (torch.rand(8, 512, generator=g, dtype=torch.float64) * 1000 - 500).to(torch.bfloat16)
+    codes, s = oracle.quantize_e4m3(x, 8, lib_path=lib)
+    top = np.abs(oracle.e4m3_values(lib_path=lib)[codes]).max(-1)
+    assert np.all((top > 224) & (top <= 448))
+    assert np.all(np.abs(x.double().numpy()).max(-1) <= 448 * s)
+    assert np.all(np.abs(x.double().numpy()).max(-1) > 224 * s)
+
+
 @pytest.mark.parametrize("fn", PINS, ids=[f.__name__ for f in PINS])
 def test_pin(fn):
     fn(None)
