@@ -82,12 +82,20 @@ struct PPCfg {
   static constexpr int kQSlot = 2 * kQTile;  // two row blocks
   // With two Q slots, a row block's O is staged in its own (finished) Q tile
   // and written by a TMA store; the slot is released once the store has read
-  // it.  An e4m3 Q tile is too small to hold the bf16 O tile.
-  static constexpr bool kTmaEpi = kQS == 2 && !QK8;
+  // it.  An e4m3 Q tile is too small to hold the bf16 O tile: there, where
+  // shared memory has room (the e4m3 Q slots take half the bytes), each row
+  // block stages O in a tile of its own (kOSep) and the Q slot is released by
+  // the MMAs as without the TMA store.
+  static constexpr int kOTile = kRows * D * 2;
+  static constexpr bool kOSep =
+      QK8 && kQS == 2 &&
+      kQS * kQSlot + kKS * kKBytes + kVS * kVBytes + 2 * kOTile + 4096 <= 227 * 1024;
+  static constexpr bool kTmaEpi = kQS == 2 && (!QK8 || kOSep);
   static constexpr int kOffQ = 0;
   static constexpr int kOffK = kOffQ + kQS * kQSlot;
   static constexpr int kOffV = kOffK + kKS * kKBytes;
-  static constexpr int kOffBar = kOffV + kVS * kVBytes;
+  static constexpr int kOffO = kOffV + kVS * kVBytes;
+  static constexpr int kOffBar = kOffO + (kOSep ? 2 * kOTile : 0);
   // k_full[KS], v_full[VS], commit ring[2][CR], p_full[2][SB], dec[2][DR],
   // q_full[QS], q_empty[QS], mma_done
   static constexpr int kNumBars = kKS + kVS + 2 * kCR + 2 * kSB + 2 * kDR + 2 * kQS + 1;
@@ -230,6 +238,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
   // variable-length batches store O row by row: a TMA store of the last row
   // block would write into the next sequence's rows
   constexpr bool kTmaEpi = C::kTmaEpi && !VARLEN;
+  constexpr bool kOSep = C::kOSep && !VARLEN;  // O staged apart from the Q slot
   constexpr int SB = C::kSB;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -293,7 +302,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
     }
     for (int s = 0; s < C::kQS; ++s) {
       mbar_init(b_q_full(s), 1);
-      mbar_init(b_q_empty(s), kTmaEpi ? 2 : 1);  // one arrival per row block's O store
+      mbar_init(b_q_empty(s), (kTmaEpi && !kOSep) ? 2 : 1);  // one arrival per row block's O store
     }
     mbar_init(b_mma_done, 1);
     for (int t = 0; t < 2; ++t)
@@ -519,7 +528,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         }
         if (!alive) break;
         // the Q slot is free once the item's last S MMA has run
-        if (!kTmaEpi && it.Tmax <= SB) mma_commit(b_q_empty(qs));
+        if ((!kTmaEpi || kOSep) && it.Tmax <= SB) mma_commit(b_q_empty(qs));
         bool started[2] = {false, false};
         for (int j = 0; alive && j < it.Tmax; ++j) {
           bool v_used = false, k_next = false;
@@ -574,7 +583,8 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           }
           if (k_next) ++kuse;
           if (v_used) ++vuse;
-          if (!kTmaEpi && j + SB + 1 == it.Tmax) mma_commit(b_q_empty(qs));  // last S MMAs issued
+          if ((!kTmaEpi || kOSep) && j + SB + 1 == it.Tmax)
+            mma_commit(b_q_empty(qs));  // last S MMAs issued
         }
         ++items;
       }
@@ -600,7 +610,8 @@ __global__ void __launch_bounds__(kPPThreads, 1)
     auto release_pending = [&]() {
       if (kTmaEpi && pend_slot >= 0) {
         bulk_wait_read_all();
-        for (int k = 0; k < pend_n; ++k) mbar_arrive(b_q_empty(pend_slot));
+        if (!kOSep)
+          for (int k = 0; k < pend_n; ++k) mbar_arrive(b_q_empty(pend_slot));
         pend_slot = -1;
       }
     };
@@ -817,7 +828,8 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         // more (its last S MMA completed before the last P*V), in the TMA
         // layout (64-column panels, 128-byte swizzle), then one thread stores
         // the tile; rows past N are clipped by the store.
-        const uint32_t stage = sQ + qs * C::kQSlot + t * C::kQTile;
+        const uint32_t stage =
+            kOSep ? sbase + C::kOffO + t * C::kOTile : sQ + qs * C::kQSlot + t * C::kQTile;
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t r[32];
@@ -981,7 +993,8 @@ int pp_launch(const PrefillLaunch& a) {
         !pp_map_e4m3(&mk, a.K, a.B * a.Hkv, a.N, D, BC) ||
         !pp_map(&mv, a.V, a.B * a.Hkv, a.N, D, BC))
       return ATTN_ERR_CUDA;
-    mo = mv;  // unused: e4m3 Q tiles cannot stage O, which is stored row by row
+    if (!C::kOSep) mo = mv;  // unused: O is stored row by row
+    else if (!pp_map(&mo, a.O, a.B * a.Hq, a.N, D, kRows)) return ATTN_ERR_CUDA;
   } else if (!pp_map(&mq, a.Q, a.B * a.Hq, a.N, D, kRows) ||
              !pp_map(&mk, a.K, a.B * a.Hkv, a.N, D, BC) ||
              !pp_map(&mv, a.V, a.B * a.Hkv, a.N, D, BC) ||
