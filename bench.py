@@ -420,7 +420,7 @@ def main():
         extras[f"{name} qk8@tau={tau}"] = entry
         del Q8, K8, Od
 
-    prefill_extra(MAIN, w, Q, K, V, math.inf, 3, 1)
+    prefill_extra(MAIN, w, Q, K, V, math.inf, max(3, args.steps // 4), 3)
     prefill_extra(MAIN, w, Q, K, V, 4.0, max(3, args.steps // 4), 2)
     if not args.quick:
         qk8_extra(MAIN, w, Q, K, V, math.inf, max(3, args.steps // 4), 2)
