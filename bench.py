@@ -393,37 +393,41 @@ def main():
                                        if ms_x >= 50.0 else None),
             "skipped_fraction": skipped, "tiles_visited": visited}
 
-    def qk8_extra(name, wl, Qd, Kd, Vd, tau, steps, warmup):
-        """The FP8 Q K^T path: e4m3 Q and K (quantised once, outside the
-        timed region; the quantiser is timed on its own), bf16 P*V."""
-        Q8, qs = bss.quantize_e4m3(Qd)
-        K8, ks = bss.quantize_e4m3(Kd)
+    def qk8_extra(name, wl, Qd, Kd, Vd, tau, steps, warmup, int8=False):
+        """The 8-bit Q K^T paths: e4m3 (or int8) Q and K, quantised once,
+        outside the timed region (the quantiser is timed on its own), bf16 P*V."""
+        quant = bss.quantize_i8 if int8 else bss.quantize_e4m3
+        prefill8 = bss.prefill_qki8 if int8 else bss.prefill_qk8
+        tag = "qki8" if int8 else "qk8"
+        Q8, qs = quant(Qd)
+        K8, ks = quant(Kd)
         Od = torch.empty_like(Qd)
-        run = lambda: bss.prefill_qk8(Q8, K8, qs, ks, Vd, wl["causal"], tau, wl["Br"], wl["Bc"], out=Od)
-        ms_x, _, _ = timed(run, steps, warmup, f"{name} qk8@tau={tau}")
-        _, mask = bss.prefill_qk8(Q8, K8, qs, ks, Vd, wl["causal"], tau, wl["Br"], wl["Bc"], out=Od,
-                                  skip_mask=True)
+        run = lambda: prefill8(Q8, K8, qs, ks, Vd, wl["causal"], tau, wl["Br"], wl["Bc"], out=Od)
+        ms_x, _, _ = timed(run, steps, warmup, f"{name} {tag}@tau={tau}")
+        _, mask = prefill8(Q8, K8, qs, ks, Vd, wl["causal"], tau, wl["Br"], wl["Bc"], out=Od,
+                           skip_mask=True)
         skipped = float((mask[mask != 2] == 1).float().mean().item())
         f = dense_flops(wl)
-        # half the dense FLOPs (Q K^T) run at the e4m3 rate, twice the bf16
+        # half the dense FLOPs (Q K^T) run at the 8-bit rate, twice the bf16
         # rate (nominal ratio); the mixed peak is 4/3 of the bf16 peak
         mixed_peak = peaks["bf16_tflops"] * 4.0 / 3.0
         entry = {"ms": ms_x, "dense_tflops": f / (ms_x * 1e-3) / 1e12,
                  "frac_of_mixed_peak": f / (ms_x * 1e-3) / 1e12 / mixed_peak,
                  "mixed_peak_tflops": mixed_peak, "skipped_fraction": skipped}
         if tau == math.inf:
-            ms_q, _, _ = timed(lambda: (bss.quantize_e4m3(Qd, out=(Q8, qs)), bss.quantize_e4m3(Kd, out=(K8, ks))),
-                               steps, warmup, f"{name} quantize")
+            ms_q, _, _ = timed(lambda: (quant(Qd, out=(Q8, qs)), quant(Kd, out=(K8, ks))),
+                               steps, warmup, f"{name} quantize {tag}")
             qbytes = (Qd.numel() + Kd.numel()) * 3  # read bf16, write e4m3
             entry["quantize_q_and_k_ms"] = ms_q
             entry["quantize_gbs"] = qbytes / (ms_q * 1e-3) / 1e9
-        extras[f"{name} qk8@tau={tau}"] = entry
+        extras[f"{name} {tag}@tau={tau}"] = entry
         del Q8, K8, Od
 
     prefill_extra(MAIN, w, Q, K, V, math.inf, max(3, args.steps // 4), 3)
     prefill_extra(MAIN, w, Q, K, V, 4.0, max(3, args.steps // 4), 2)
     if not args.quick:
         qk8_extra(MAIN, w, Q, K, V, math.inf, max(3, args.steps // 4), 2)
+        qk8_extra(MAIN, w, Q, K, V, math.inf, max(3, args.steps // 4), 2, int8=True)
     del Q, K, V, O
     torch.cuda.empty_cache()
 
@@ -497,6 +501,7 @@ def main():
             if name == "llama3_8b_causal_N8192":
                 for tau in (math.inf, 4.0):
                     qk8_extra(name, wl, Qd, Kd2, Vd2, tau, steps, 1)
+                qk8_extra(name, wl, Qd, Kd2, Vd2, math.inf, steps, 1, int8=True)
             del Qd, Kd2, Vd2
             torch.cuda.empty_cache()
     if rank == 0:

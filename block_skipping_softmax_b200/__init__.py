@@ -20,7 +20,8 @@ import os
 __all__ = [
     "AttnError", "lib", "attn_prefill", "attn_prefill_ex", "attn_prefill_host", "prefill_host",
     "attn_prefill_varlen", "prefill_varlen", "attn_quantize_e4m3", "quantize_e4m3",
-    "attn_prefill_qk8", "prefill_qk8", "attn_decode", "attn_decode_ex",
+    "attn_prefill_qk8", "prefill_qk8", "attn_quantize_i8", "quantize_i8", "attn_prefill_qki8",
+    "prefill_qki8", "attn_decode", "attn_decode_ex",
     "attn_decode_noalloc", "attn_decode_rule", "attn_decode_paged", "decode_paged", "RULE_GROUP", "RULE_PER_HEAD", "RULE_SINK_SEED",
     "attn_decode_split_len", "attn_decode_tile", "attn_decode_workspace_bytes",
     "attn_set_stream", "attn_sync_status", "attn_last_timeout_site", "attn_set_wait_limit_ms",
@@ -58,6 +59,8 @@ def lib() -> ctypes.CDLL:
         "attn_prefill_varlen": (ci, [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, cf, ci, ci, vp, vp]),
         "attn_quantize_e4m3": (ci, [vp, vp, vp, ctypes.c_longlong, ctypes.c_longlong, vp]),
         "attn_prefill_qk8": (ci, [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, ci, vp, vp]),
+        "attn_quantize_i8": (ci, [vp, vp, vp, ctypes.c_longlong, ctypes.c_longlong, vp]),
+        "attn_prefill_qki8": (ci, [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, ci, vp, vp]),
         "attn_decode": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf]),
         "attn_decode_ex": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, vp, vp, vp, sz]),
         "attn_decode_noalloc": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, cf, vp, vp]),
@@ -115,6 +118,16 @@ def attn_prefill_qk8(Q8, K8, q_scales, k_scales, V, O, B, Hq, Hkv, N, d, causal,
                      skip_mask=None) -> int:
     return lib().attn_prefill_qk8(Q8, K8, q_scales, k_scales, V, O, B, Hq, Hkv, N, d, int(causal),
                                   float(tau), Br, Bc, stream, skip_mask)
+
+
+def attn_quantize_i8(x, q, scales, groups, group_elems, stream=None) -> int:
+    return lib().attn_quantize_i8(x, q, scales, int(groups), int(group_elems), stream)
+
+
+def attn_prefill_qki8(Q8, K8, q_scales, k_scales, V, O, B, Hq, Hkv, N, d, causal, tau, Br, Bc, stream=None,
+                      skip_mask=None) -> int:
+    return lib().attn_prefill_qki8(Q8, K8, q_scales, k_scales, V, O, B, Hq, Hkv, N, d, int(causal),
+                                   float(tau), Br, Bc, stream, skip_mask)
 
 
 def attn_decode(q, K, V, o, B, Hq, Hkv, L, d, tau) -> int:
@@ -256,21 +269,35 @@ def quantize_e4m3(x, out=None, stream=None):
     """e4m3 codes (uint8, x's shape) and one power-of-two scale per head slab
     (float32 [B, H]) of a contiguous bf16 CUDA tensor x [B, H, N, d].
     ``out`` = (codes, scales) writes into existing tensors."""
+    return _quantize(x, out, stream, int8=False)
+
+
+def quantize_i8(x, out=None, stream=None):
+    """int8 codes (int8, x's shape) and one power-of-two scale per head slab
+    (float32 [B, H]) of a contiguous bf16 CUDA tensor x [B, H, N, d]."""
+    return _quantize(x, out, stream, int8=True)
+
+
+def _quantize(x, out, stream, int8):
     import torch
 
+    code_dtype = torch.int8 if int8 else torch.uint8
+    what = "quantize_i8" if int8 else "quantize_e4m3"
+
     if x.dtype != torch.bfloat16 or not x.is_cuda or not x.is_contiguous() or x.dim() != 4:
-        raise AttnError(1, "quantize_e4m3 (x must be a contiguous 4-d bf16 CUDA tensor)")
+        raise AttnError(1, f"{what} (x must be a contiguous 4-d bf16 CUDA tensor)")
     B, H, N, d = x.shape
     if out is not None:
         q, scales = out
-        if (q.dtype != torch.uint8 or q.shape != x.shape or not q.is_contiguous() or
+        if (q.dtype != code_dtype or q.shape != x.shape or not q.is_contiguous() or
                 scales.dtype != torch.float32 or scales.numel() != B * H or not scales.is_contiguous()):
-            raise AttnError(1, "quantize_e4m3 (out must be uint8 codes of x's shape and float32 [B, H])")
+            raise AttnError(1, f"{what} (out must be {code_dtype} codes of x's shape and float32 [B, H])")
     else:
-        q = torch.empty(x.shape, dtype=torch.uint8, device=x.device)
+        q = torch.empty(x.shape, dtype=code_dtype, device=x.device)
         scales = torch.empty(B, H, dtype=torch.float32, device=x.device)
-    _check(attn_quantize_e4m3(x.data_ptr(), q.data_ptr(), scales.data_ptr(), B * H, N * d,
-                              _stream_ptr(stream)), "attn_quantize_e4m3")
+    fn = attn_quantize_i8 if int8 else attn_quantize_e4m3
+    _check(fn(x.data_ptr(), q.data_ptr(), scales.data_ptr(), B * H, N * d, _stream_ptr(stream)),
+           "attn_" + what)
     return q, scales
 
 
@@ -278,26 +305,40 @@ def prefill_qk8(Q8, K8, q_scales, k_scales, V, causal: bool, tau: float = math.i
                 Bc: int = 128, out=None, skip_mask: bool = False, stream=None):
     """Prefill with e4m3 Q8 [B,Hq,N,d], K8 [B,Hkv,N,d] (uint8 codes from
     quantize_e4m3), float32 scales [B,Hq] / [B,Hkv], and bf16 V."""
+    return _prefill_8bit(Q8, K8, q_scales, k_scales, V, causal, tau, Br, Bc, out, skip_mask, stream, False)
+
+
+def prefill_qki8(Q8, K8, q_scales, k_scales, V, causal: bool, tau: float = math.inf, Br: int = 128,
+                 Bc: int = 128, out=None, skip_mask: bool = False, stream=None):
+    """Prefill with int8 Q8 [B,Hq,N,d], K8 [B,Hkv,N,d] (codes from
+    quantize_i8), float32 scales [B,Hq] / [B,Hkv], and bf16 V."""
+    return _prefill_8bit(Q8, K8, q_scales, k_scales, V, causal, tau, Br, Bc, out, skip_mask, stream, True)
+
+
+def _prefill_8bit(Q8, K8, q_scales, k_scales, V, causal, tau, Br, Bc, out, skip_mask, stream, int8):
     import torch
 
+    what = "prefill_qki8" if int8 else "prefill_qk8"
+    code_dtype = torch.int8 if int8 else torch.uint8
     B, Hq, N, d = Q8.shape
     Hkv = K8.shape[1]
     for t in (Q8, K8):
-        if t.dtype != torch.uint8 or not t.is_cuda or not t.is_contiguous():
-            raise AttnError(1, "prefill_qk8 (Q8, K8 must be contiguous uint8 CUDA tensors)")
+        if t.dtype != code_dtype or not t.is_cuda or not t.is_contiguous():
+            raise AttnError(1, f"{what} (Q8, K8 must be contiguous {code_dtype} CUDA tensors)")
     for t in (q_scales, k_scales):
         if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
-            raise AttnError(1, "prefill_qk8 (scales must be contiguous float32 CUDA tensors)")
+            raise AttnError(1, f"{what} (scales must be contiguous float32 CUDA tensors)")
     if V.dtype != torch.bfloat16 or not V.is_cuda or not V.is_contiguous():
-        raise AttnError(1, "prefill_qk8 (V must be a contiguous bf16 CUDA tensor)")
+        raise AttnError(1, f"{what} (V must be a contiguous bf16 CUDA tensor)")
     O = out if out is not None else torch.empty(Q8.shape, dtype=torch.bfloat16, device=Q8.device)
     mask = None
     if skip_mask:
         mask = torch.empty(B, Hq, -(-N // Br), -(-N // Bc), dtype=torch.uint8, device=Q8.device)
-    st = attn_prefill_qk8(Q8.data_ptr(), K8.data_ptr(), q_scales.data_ptr(), k_scales.data_ptr(),
-                          V.data_ptr(), O.data_ptr(), B, Hq, Hkv, N, d, causal, tau, Br, Bc,
-                          _stream_ptr(stream), mask.data_ptr() if mask is not None else None)
-    _check(st, "attn_prefill_qk8")
+    fn = attn_prefill_qki8 if int8 else attn_prefill_qk8
+    st = fn(Q8.data_ptr(), K8.data_ptr(), q_scales.data_ptr(), k_scales.data_ptr(),
+            V.data_ptr(), O.data_ptr(), B, Hq, Hkv, N, d, causal, tau, Br, Bc,
+            _stream_ptr(stream), mask.data_ptr() if mask is not None else None)
+    _check(st, "attn_" + what)
     return (O, mask) if skip_mask else O
 
 

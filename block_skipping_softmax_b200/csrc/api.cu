@@ -172,9 +172,9 @@ int attn_prefill_varlen(const void* Q, const void* K, const void* V, void* O,
   return bss::launch_prefill_pp(a);
 }
 
-int attn_prefill_qk8(const void* Q8, const void* K8, const float* q_scales, const float* k_scales,
-                     const void* V, void* O, int B, int Hq, int Hkv, int N, int d, int causal,
-                     float tau, int Br, int Bc, void* stream, uint8_t* skip_mask) {
+static int prefill_8bit(const void* Q8, const void* K8, const float* q_scales, const float* k_scales,
+                        const void* V, void* O, int B, int Hq, int Hkv, int N, int d, int causal, float tau,
+                        int Br, int Bc, void* stream, uint8_t* skip_mask, int format) {
   if (!q_scales || !k_scales) return ATTN_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(q_scales) & 3u) || (reinterpret_cast<uintptr_t>(k_scales) & 3u))
     return ATTN_ERR_INVALID_ARG;
@@ -206,7 +206,22 @@ int attn_prefill_qk8(const void* Q8, const void* K8, const float* q_scales, cons
   a.stream = static_cast<cudaStream_t>(stream);
   a.q_scales = q_scales;
   a.k_scales = k_scales;
+  a.qk_format = format;
   return bss::launch_prefill_pp(a);
+}
+
+int attn_prefill_qk8(const void* Q8, const void* K8, const float* q_scales, const float* k_scales,
+                     const void* V, void* O, int B, int Hq, int Hkv, int N, int d, int causal,
+                     float tau, int Br, int Bc, void* stream, uint8_t* skip_mask) {
+  return prefill_8bit(Q8, K8, q_scales, k_scales, V, O, B, Hq, Hkv, N, d, causal, tau, Br, Bc, stream,
+                      skip_mask, 1);
+}
+
+int attn_prefill_qki8(const void* Q8, const void* K8, const float* q_scales, const float* k_scales,
+                      const void* V, void* O, int B, int Hq, int Hkv, int N, int d, int causal,
+                      float tau, int Br, int Bc, void* stream, uint8_t* skip_mask) {
+  return prefill_8bit(Q8, K8, q_scales, k_scales, V, O, B, Hq, Hkv, N, d, causal, tau, Br, Bc, stream,
+                      skip_mask, 2);
 }
 
 int attn_prefill(const void* Q, const void* K, const void* V, void* O, int B, int Hq, int Hkv,

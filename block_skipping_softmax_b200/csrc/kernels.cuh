@@ -33,6 +33,7 @@ struct PrefillLaunch {
   // (k_scales[b*Hkv+h]); V and O stay bf16
   const float* q_scales;
   const float* k_scales;
+  int qk_format;  // with q_scales: 1 e4m3, 2 signed int8
 };
 
 int launch_prefill(const PrefillLaunch& a);     // one row block per CTA (any Br)

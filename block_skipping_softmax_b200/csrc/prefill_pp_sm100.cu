@@ -47,6 +47,7 @@ constexpr int kPPThreads = 384;
 constexpr int kPPRegs = 168;  // registers per thread at launch (checked on the host)
 constexpr int kRows = 128;    // rows per tile (row block)
 constexpr int kDR = 4;        // decision ring
+constexpr float kI2FOffset = 12582912.f;  // 1.5 * 2^23: int32 scores as fp32 by one integer add
 constexpr int kCR = 16;       // commit ring per row block (waiters lag by at most ~6)
 constexpr float kRescale = 8.0f;  // lazy rescale threshold (log2 units)
 // Which of the 16 column pairs of each 32-column chunk take the polynomial
@@ -224,7 +225,9 @@ struct Pending3 {
 
 }  // namespace
 
-template <int D, int BC, bool CAUSAL, bool VARLEN, bool QK8>
+// QKT: Q K^T operand format, 0 bf16, 1 e4m3 (f32 scores), 2 signed int8
+// (int32 scores)
+template <int D, int BC, bool CAUSAL, bool VARLEN, int QKT>
 __global__ void __launch_bounds__(kPPThreads, 1)
     prefill_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -234,6 +237,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                       unsigned long long wait_limit_ns, const int* __restrict__ cu_seqlens,
                       int total, const float* __restrict__ q_scales,
                       const float* __restrict__ k_scales) {
+  constexpr bool QK8 = QKT != 0;
   using C = PPCfg<D, BC, QK8>;
   // variable-length batches store O row by row: a TMA store of the last row
   // block would write into the next sequence's rows
@@ -468,8 +472,9 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         mbar_drain(b_v_full(t % C::kVS), (t / C::kVS) & 1, wait_limit_ns);
     } else if (warp == 1 && lane == 0) {
       // ---------------------------------------------------- MMA issuer
-      constexpr uint32_t idS =
-          QK8 ? idesc_e4m3_f32(kRows, BC) : idesc_bf16_f32(kRows, BC, false, false);
+      constexpr uint32_t idS = QKT == 2   ? idesc_s8_s32(kRows, BC)
+                               : QKT == 1 ? idesc_e4m3_f32(kRows, BC)
+                                          : idesc_bf16_f32(kRows, BC, false, false);
       constexpr uint32_t idPV = idesc_bf16_f32(kRows, D, false, true);
       int kuse = 0, vuse = 0, items = 0;
       int pc[2] = {0, 0}, dc[2] = {0, 0}, sq[2] = {0, 0}, cmc[2] = {0, 0};
@@ -487,7 +492,10 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         for (int kk = 0; kk < C::kSSteps; ++kk) {  // 32 bytes of the reduction each
           const uint32_t oq = ((kk >> 2) * C::kQPanel + (kk & 3) * 32) >> 4;
           const uint32_t ok_ = ((kk >> 2) * C::kKVPanel + (kk & 3) * 32) >> 4;
-          if constexpr (QK8)
+          if constexpr (QKT == 2)
+            mma_ss_i8(tS(t, buf), desc_join(a0 + oq, kHi), desc_join(b0 + ok_, kHi), idS,
+                      kk > 0 ? 1u : 0u);
+          else if constexpr (QKT == 1)
             mma_ss_f8(tS(t, buf), desc_join(a0 + oq, kHi), desc_join(b0 + ok_, kHi), idS,
                       kk > 0 ? 1u : 0u);
           else
@@ -650,6 +658,14 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           tc_fence_after();
           tmem_ld_row<BC>(tS(t, sb) + lane_off, u);
           tmem_wait_ld();
+          if constexpr (QKT == 2) {
+            // int32 scores (|i| < 2^22 for 8-bit operands, d <= 128) become
+            // the fp32 values 1.5 * 2^23 + i by one integer add to the bit
+            // pattern of 1.5 * 2^23; the offset is taken out of the max below
+            // and folded into the exponent's bias
+#pragma unroll
+            for (int c = 0; c < BC; ++c) u[c] += 0x4B400000u;
+          }
           // last visible column of this row in tile j (-1: none); one integer
           // limit keeps the masking to a compare-select per column
           const int key0 = j * BC;
@@ -667,7 +683,9 @@ __global__ void __launch_bounds__(kPPThreads, 1)
 #pragma unroll
             for (int k = 0; k < 4; ++k)
               m4[k] = fmax3(m4[k], __uint_as_float(u[c + 2 * k]), __uint_as_float(u[c + 2 * k + 1]));
-          mt = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * sl2;  // log2 units; -inf stays -inf
+          const float mraw = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
+          // log2 units; -inf stays -inf; the int8 offset comes out exactly
+          mt = (QKT == 2 ? mraw - kI2FOffset : mraw) * sl2;
         }
         // ---- skip test: every row of this row block must have mt < m - tau.
         // Each warp publishes its own verdict (all its rows pass, or not) and
@@ -740,7 +758,9 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         // P = 2^(s*scale - m_ref): one packed FFMA per pair, two ex2, one
         // pack to bf16 for the P*V MMA; the row sum adds the fp32 pair with
         // one packed add (four independent chains)
-        const float neg_m = row_valid ? -m_ref : 0.f;  // invalid rows: all scores -inf -> P = 0
+        // invalid rows: all scores -inf -> P = 0; int8 scores carry the
+        // offset 1.5 * 2^23, taken out here
+        const float neg_m = (row_valid ? -m_ref : 0.f) - (QKT == 2 ? kI2FOffset * sl2 : 0.f);
         const float2 sc2 = make_float2(sl2, sl2);
         const float2 nm2 = make_float2(neg_m, neg_m);
         float2 rs2[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
@@ -956,10 +976,11 @@ bool pp_map_thd(CUtensorMap* m, const void* base, int H, int tokens, int D, int 
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int BC, bool CAUSAL, bool VARLEN, bool QK8>
+template <int D, int BC, bool CAUSAL, bool VARLEN, int QKT>
 int pp_launch(const PrefillLaunch& a) {
+  constexpr bool QK8 = QKT != 0;
   using C = PPCfg<D, BC, QK8>;
-  auto kern = prefill_pp_kernel<D, BC, CAUSAL, VARLEN, QK8>;
+  auto kern = prefill_pp_kernel<D, BC, CAUSAL, VARLEN, QKT>;
   static uint64_t ready = 0;  // one bit per device: attributes set and checked
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return ATTN_ERR_CUDA;
@@ -1014,21 +1035,27 @@ int pp_launch(const PrefillLaunch& a) {
 template <int D, int BC>
 int pp_launch_c(const PrefillLaunch& a) {
   if (a.cu_seqlens)
-    return a.causal ? pp_launch<D, BC, true, true, false>(a) : pp_launch<D, BC, false, true, false>(a);
-  return a.causal ? pp_launch<D, BC, true, false, false>(a) : pp_launch<D, BC, false, false, false>(a);
+    return a.causal ? pp_launch<D, BC, true, true, 0>(a) : pp_launch<D, BC, false, true, 0>(a);
+  return a.causal ? pp_launch<D, BC, true, false, 0>(a) : pp_launch<D, BC, false, false, 0>(a);
 }
 
 }  // namespace
 
 int launch_prefill_pp(const PrefillLaunch& a) {
   if (a.Br != 128) return ATTN_ERR_INVALID_ARG;
-  if (a.q_scales) {  // e4m3 Q and K: d = 128, fixed-length batches
+  if (a.q_scales) {  // 8-bit Q and K: d = 128, fixed-length batches
     if (a.d != 128 || a.cu_seqlens) return ATTN_ERR_INVALID_ARG;
-    if (a.Bc == 64)
-      return a.causal ? pp_launch<128, 64, true, false, true>(a)
-                      : pp_launch<128, 64, false, false, true>(a);
-    return a.causal ? pp_launch<128, 128, true, false, true>(a)
-                    : pp_launch<128, 128, false, false, true>(a);
+    if (a.qk_format == 1) {
+      if (a.Bc == 64)
+        return a.causal ? pp_launch<128, 64, true, false, 1>(a) : pp_launch<128, 64, false, false, 1>(a);
+      return a.causal ? pp_launch<128, 128, true, false, 1>(a) : pp_launch<128, 128, false, false, 1>(a);
+    }
+    if (a.qk_format == 2) {
+      if (a.Bc == 64)
+        return a.causal ? pp_launch<128, 64, true, false, 2>(a) : pp_launch<128, 64, false, false, 2>(a);
+      return a.causal ? pp_launch<128, 128, true, false, 2>(a) : pp_launch<128, 128, false, false, 2>(a);
+    }
+    return ATTN_ERR_INVALID_ARG;
   }
   if (a.d == 128) return a.Bc == 64 ? pp_launch_c<128, 64>(a) : pp_launch_c<128, 128>(a);
   if (a.d == 64) return a.Bc == 64 ? pp_launch_c<64, 64>(a) : pp_launch_c<64, 128>(a);

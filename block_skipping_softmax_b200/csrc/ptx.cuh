@@ -302,6 +302,13 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_ma
 
 // Instruction descriptor, kind::f8f6f4 with e4m3 A/B (format code 0 in the
 // A and B fields) and fp32 accumulation; both operands K-major.
+// kind::i8: signed int8 A and B, int32 accumulator (c format 2 = S32,
+// a/b format 1 = signed 8-bit), both K-major
+__device__ __forceinline__ void mma_ss_i8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t accumulate) {
+  asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\ttcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),"l"(a_desc),"l"(b_desc),"r"(idesc),"r"(accumulate):"memory");}
+__host__ __device__ constexpr uint32_t idesc_s8_s32(int M, int N) {
+  return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);}
 __host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
   return (1u << 4)                                // D format: f32
          | (static_cast<uint32_t>(N >> 3) << 17)  // N / 8

@@ -1,15 +1,18 @@
-// e4m3 quantisation of Q or K for the FP8 QK^T prefill path ("Accelerating
-// Long-Context Inference with Skip Softmax in NVIDIA TensorRT-LLM": the skip
-// test runs on the raw Q K^T scores, which may come from lower-precision
-// operands; the page names FP8 attention as the path it combines with).
+// 8-bit quantisation of Q or K for the low-precision Q K^T prefill paths
+// ("Accelerating Long-Context Inference with Skip Softmax in NVIDIA
+// TensorRT-LLM": the skip test runs on the raw Q K^T scores, which may come
+// from lower-precision operands; the page names FP8 attention as the path it
+// combines with; "TurboAttention", Technical Deep Dive: integer Q K^T inside
+// the tile loop).
 //
 // A tensor is cut into `groups` contiguous groups (one head slab [N, d] each
 // for the prefill layouts).  Each group gets one power-of-two scale s, the
-// smallest with max|x| <= 448 s (448 is the largest finite e4m3 value), and
-// every element becomes e4m3(x / s), rounded to nearest, ties to even.
-// Because s is a power of two, x / s is exact, and the dequantised value
-// e4m3(x / s) * s (three mantissa bits) is exact in bf16: a bf16 reference fed
-// the dequantised tensors sees exactly the operands the FP8 MMAs see.
+// smallest with max|x| <= M s, where M is the format's largest value (448
+// for e4m3, 127 for int8), and every element becomes e4m3(x / s) or the
+// integer nearest x / s, ties to even.  Because s is a power of two, x / s is
+// exact, and the dequantised value code * s (three mantissa bits, or an
+// integer of at most 7 bits) is exact in bf16: a bf16 reference fed the
+// dequantised tensors sees exactly the operands the 8-bit MMAs see.
 //
 // Three launches, all bound by HBM: a per-group max of |x| (one atomic per
 // block, on the bit pattern: non-negative floats order like their bits),
@@ -68,11 +71,12 @@ __global__ void __launch_bounds__(kThreads) amax_kernel(const uint4* __restrict_
 }
 
 // In place: the max bits of each group become its scale.  max|x| = f 2^e with
-// f in [0.5, 1), and 448 = 0.875 * 2^9, so max|x| <= 448 * 2^k holds first at
-// k = e - 9 when f <= 0.875, else at k = e - 8.  k is held at -126 or above,
-// so that 1/s stays finite (only groups whose max is below 2^-117 notice).
-// A zero group gets scale 1; a group holding inf or NaN gets NaN.
-__global__ void scale_kernel(float* __restrict__ scales, long long groups) {
+// f in [0.5, 1), and M = m 2^p with m in [0.5, 1) (448 = 0.875 * 2^9,
+// 127 = (127/128) * 2^7), so max|x| <= M 2^k holds first at k = e - p when
+// f <= m, else at k = e - p + 1.  k is held at -126 or above, so that 1/s
+// stays finite (only groups whose max is below about 2^-118 notice).  A zero
+// group gets scale 1; a group holding inf or NaN gets NaN.
+__global__ void scale_kernel(float* __restrict__ scales, long long groups, float m, int p) {
   const long long g = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (g >= groups) return;
   const uint32_t bits = __float_as_uint(scales[g]);
@@ -84,11 +88,12 @@ __global__ void scale_kernel(float* __restrict__ scales, long long groups) {
   } else {
     int e = 0;
     const float f = frexpf(__uint_as_float(bits), &e);
-    s = ldexpf(1.f, max(f <= 0.875f ? e - 9 : e - 8, -126));
+    s = ldexpf(1.f, max(f <= m ? e - p : e - p + 1, -126));
   }
   scales[g] = s;
 }
 
+template <bool INT8>
 __global__ void __launch_bounds__(kThreads) convert_kernel(const uint4* __restrict__ x,
                                                            uint4* __restrict__ q,
                                                            const float* __restrict__ scales,
@@ -113,10 +118,17 @@ __global__ void __launch_bounds__(kThreads) convert_kernel(const uint4* __restri
       const float e1 = __uint_as_float(w[2 * k] & 0xffff0000u) * inv;
       const float e2 = __uint_as_float(w[2 * k + 1] << 16) * inv;
       const float e3 = __uint_as_float(w[2 * k + 1] & 0xffff0000u) * inv;
-      uint16_t lo, hi;  // cvt packs its first source into the upper byte
-      asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(e1), "f"(e0));
-      asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(e3), "f"(e2));
-      out[k] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+      if constexpr (INT8) {  // nearest integer, ties to even (|x / s| <= 127)
+        const int i0 = __float2int_rn(e0), i1 = __float2int_rn(e1);
+        const int i2 = __float2int_rn(e2), i3 = __float2int_rn(e3);
+        out[k] = (static_cast<uint32_t>(i0) & 0xffu) | ((static_cast<uint32_t>(i1) & 0xffu) << 8) |
+                 ((static_cast<uint32_t>(i2) & 0xffu) << 16) | (static_cast<uint32_t>(i3) << 24);
+      } else {
+        uint16_t lo, hi;  // cvt packs its first source into the upper byte
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(lo) : "f"(e1), "f"(e0));
+        asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(hi) : "f"(e3), "f"(e2));
+        out[k] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+      }
     }
     dst[v] = make_uint4(out[0], out[1], out[2], out[3]);
   }
@@ -124,12 +136,8 @@ __global__ void __launch_bounds__(kThreads) convert_kernel(const uint4* __restri
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-}  // namespace
-
-extern "C" {
-
-int attn_quantize_e4m3(const void* x, void* q, float* scales, long long groups,
-                       long long group_elems, void* stream) {
+int quantize(const void* x, void* q, float* scales, long long groups, long long group_elems,
+             void* stream, bool int8) {
   if (!x || !q || !scales || groups <= 0 || group_elems <= 0) return ATTN_ERR_INVALID_ARG;
   if (group_elems % 16 != 0 || !aligned16(x) || !aligned16(q) ||
       (reinterpret_cast<uintptr_t>(scales) & 3u))
@@ -147,10 +155,31 @@ int attn_quantize_e4m3(const void* x, void* q, float* scales, long long groups,
     return ATTN_ERR_CUDA;
   amax_kernel<<<grid, kThreads, 0, s>>>(static_cast<const uint4*>(x),
                                         reinterpret_cast<unsigned int*>(scales), vpg, bpg);
-  scale_kernel<<<static_cast<unsigned int>((groups + 255) / 256), 256, 0, s>>>(scales, groups);
-  convert_kernel<<<grid, kThreads, 0, s>>>(static_cast<const uint4*>(x), static_cast<uint4*>(q),
-                                           scales, vpg, bpg);
+  const unsigned int sgrid = static_cast<unsigned int>((groups + 255) / 256);
+  if (int8) {
+    scale_kernel<<<sgrid, 256, 0, s>>>(scales, groups, 127.f / 128.f, 7);
+    convert_kernel<true><<<grid, kThreads, 0, s>>>(static_cast<const uint4*>(x),
+                                                   static_cast<uint4*>(q), scales, vpg, bpg);
+  } else {
+    scale_kernel<<<sgrid, 256, 0, s>>>(scales, groups, 0.875f, 9);
+    convert_kernel<false><<<grid, kThreads, 0, s>>>(static_cast<const uint4*>(x),
+                                                    static_cast<uint4*>(q), scales, vpg, bpg);
+  }
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_quantize_e4m3(const void* x, void* q, float* scales, long long groups,
+                       long long group_elems, void* stream) {
+  return quantize(x, q, scales, groups, group_elems, stream, false);
+}
+
+int attn_quantize_i8(const void* x, void* q, float* scales, long long groups,
+                     long long group_elems, void* stream) {
+  return quantize(x, q, scales, groups, group_elems, stream, true);
 }
 
 }  // extern "C"

@@ -138,6 +138,27 @@ ATTN_API int attn_prefill_qk8(const void* Q8, const void* K8, const float* q_sca
                               void* stream, uint8_t* skip_mask);
 
 /*
+ * int8 quantisation (for attn_prefill_qki8): as attn_quantize_e4m3, with the
+ * scale s = 2^k, k the smallest integer >= -126 such that max|x| <= 127 * 2^k,
+ * and q[i] = the integer nearest x[i] / s, ties to even, as a signed byte
+ * (|q| <= 127).  q * s is exactly representable in bf16.  Same arguments,
+ * ownership and errors as attn_quantize_e4m3.
+ */
+ATTN_API int attn_quantize_i8(const void* x, void* q, float* scales, long long groups,
+                              long long group_elems, void* stream);
+
+/*
+ * Prefill with S = Q K^T from signed int8 operands on the tensor cores (kind
+ * i8, int32 accumulation, exact); P*V stays bf16.  Q8 and K8 as written by
+ * attn_quantize_i8 with one group per head slab; otherwise as
+ * attn_prefill_qk8 (d = 128 and Br = 128 only, same errors).
+ */
+ATTN_API int attn_prefill_qki8(const void* Q8, const void* K8, const float* q_scales,
+                               const float* k_scales, const void* V, void* O, int B, int Hq,
+                               int Hkv, int N, int d, int causal, float tau, int Br, int Bc,
+                               void* stream, uint8_t* skip_mask);
+
+/*
  * Prefill with the inputs and the output in host memory: the batch is cut
  * into chunks of `chunk` sequences (0: B/8 rounded up) that flow through two
  * library-owned device buffer sets on two library streams, so the copy of

@@ -70,6 +70,9 @@ def _load(path: str | None = None):
     lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
     lib.oracle_quantize_e4m3.restype = ci
     lib.oracle_quantize_e4m3.argtypes = [u16p, ctypes.c_int64, ctypes.c_int64, u8p, f64p]
+    lib.oracle_quantize_i8.restype = ci
+    lib.oracle_quantize_i8.argtypes = [u16p, ctypes.c_int64, ctypes.c_int64,
+                                       ctypes.POINTER(ctypes.c_int8), f64p]
     if path is None:
         _lib = lib
     return lib
@@ -193,3 +196,24 @@ def dequantize_e4m3(codes: np.ndarray, scales: np.ndarray, lib_path: str | None 
     """fp64 values code * scale, one scale per equal contiguous group."""
     vals = e4m3_values(lib_path)[codes.reshape(scales.size, -1)]
     return (vals * scales[:, None]).reshape(codes.shape)
+
+
+def quantize_i8(x, groups: int, lib_path: str | None = None):
+    """int8 codes (x's shape) and fp64 power-of-two scales [groups] of a bf16
+    tensor cut into ``groups`` equal contiguous groups."""
+    xb = _bits(x)
+    n = xb.size
+    if groups <= 0 or n % groups:
+        raise ValueError("quantize_i8: the element count must split into equal groups")
+    codes = np.empty(xb.shape, dtype=np.int8)
+    scales = np.empty(groups)
+    st = _load(lib_path).oracle_quantize_i8(_p(xb, ctypes.c_uint16), groups, n // groups,
+                                            _p(codes, ctypes.c_int8), _p(scales, ctypes.c_double))
+    if st != 0:
+        raise ValueError(f"oracle_quantize_i8 failed with status {st}")
+    return codes, scales
+
+
+def dequantize_i8(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """fp64 values code * scale, one scale per equal contiguous group."""
+    return (codes.reshape(scales.size, -1).astype(np.float64) * scales[:, None]).reshape(codes.shape)

@@ -515,3 +515,59 @@ int oracle_quantize_e4m3(const uint16_t *x, int64_t groups, int64_t group_elems,
     }
     return ORACLE_OK;
 }
+
+/*
+ * int8 quantisation for the integer Q K^T path ("TurboAttention", Technical
+ * Deep Dive, quantises Q and K to integers inside the tile loop; the scale
+ * rule is this library's own, stated here in full): s = 2^k with k the
+ * smallest integer >= -126 such that max|x| <= 127 * 2^k (s = 1 for a group of
+ * zeros, NaN for a group holding inf or NaN); code_i = the integer nearest
+ * x_i / s, ties to the even integer, as a two's-complement byte (|code| <= 127).
+ */
+static int8_t nearest_int_even(double y)
+{
+    const double f = floor(y);
+    const double r = y - f;  /* exact: y has few significant bits */
+    double n;
+    if (r < 0.5)
+        n = f;
+    else if (r > 0.5)
+        n = f + 1.0;
+    else
+        n = (fmod(f, 2.0) == 0.0) ? f : f + 1.0;
+    return (int8_t)n;
+}
+
+int oracle_quantize_i8(const uint16_t *x, int64_t groups, int64_t group_elems, int8_t *q,
+                       double *scales)
+{
+    if (!x || !q || !scales || groups <= 0 || group_elems <= 0)
+        return ORACLE_BAD_ARG;
+    for (int64_t g = 0; g < groups; ++g) {
+        const uint16_t *xg = x + g * group_elems;
+        double amax = 0.0;
+        int finite = 1;
+        for (int64_t i = 0; i < group_elems; ++i) {
+            const double v = widen_bf16(xg[i]);
+            if (!isfinite(v))
+                finite = 0;
+            else if (fabs(v) > amax)
+                amax = fabs(v);
+        }
+        double s;
+        if (!finite) {
+            s = NAN;
+        } else if (amax == 0.0) {
+            s = 1.0;
+        } else {
+            int k = -126;
+            while (amax > ldexp(127.0, k))
+                ++k;
+            s = ldexp(1.0, k);
+        }
+        scales[g] = s;
+        for (int64_t i = 0; i < group_elems; ++i)
+            q[g * group_elems + i] = finite ? nearest_int_even(widen_bf16(xg[i]) / s) : 0;
+    }
+    return ORACLE_OK;
+}

@@ -64,21 +64,25 @@ def test_prefill_writes_only_its_outputs(Br, Bc, causal, tau):
     assert torch.equal(gm.inner.view(B, Hq, n_rb, n_t), ref_m)
 
 
+@pytest.mark.parametrize("int8", [False, True])
 @pytest.mark.parametrize("Bc", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
-def test_prefill_qk8_writes_only_its_outputs(Bc, causal):
+def test_prefill_qk8_writes_only_its_outputs(Bc, causal, int8):
     B, Hq, Hkv, N, d = 2, 4, 2, 333, 128
     Q, K, V = inputs.prefill_inputs(B, Hq, Hkv, N, d, seed=53, q_sigma=2.0, q_u=8.0, sink_scale=6.0)
-    Q8, qs = bss.quantize_e4m3(Q.cuda())
-    K8, ks = bss.quantize_e4m3(K.cuda())
+    quant = bss.quantize_i8 if int8 else bss.quantize_e4m3
+    Q8, qs = quant(Q.cuda())
+    K8, ks = quant(K.cuda())
     Vd = V.cuda()
-    ref_o, ref_m = bss.prefill_qk8(Q8, K8, qs, ks, Vd, causal, 2.0, 128, Bc, skip_mask=True)
+    run = bss.prefill_qki8 if int8 else bss.prefill_qk8
+    ref_o, ref_m = run(Q8, K8, qs, ks, Vd, causal, 2.0, 128, Bc, skip_mask=True)
     n_rb, n_t = -(-N // 128), -(-N // Bc)
     go = Guarded(B * Hq * N * d * 2)
     gm = Guarded(B * Hq * n_rb * n_t)
-    st = bss.attn_prefill_qk8(Q8.data_ptr(), K8.data_ptr(), qs.data_ptr(), ks.data_ptr(), Vd.data_ptr(),
-                              go.ptr(), B, Hq, Hkv, N, d, causal, 2.0, 128, Bc,
-                              torch.cuda.current_stream().cuda_stream, gm.ptr())
+    raw = bss.attn_prefill_qki8 if int8 else bss.attn_prefill_qk8
+    st = raw(Q8.data_ptr(), K8.data_ptr(), qs.data_ptr(), ks.data_ptr(), Vd.data_ptr(),
+             go.ptr(), B, Hq, Hkv, N, d, causal, 2.0, 128, Bc,
+             torch.cuda.current_stream().cuda_stream, gm.ptr())
     assert st == 0
     assert bss.attn_sync_status() == 0
     assert go.intact() and gm.intact()

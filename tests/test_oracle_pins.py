@@ -561,6 +561,51 @@ def pin_e4m3_scale_rule(lib):
     assert np.all(np.abs(x.double().numpy()).max(-1) > 224 * s)
 
 
+@pin
+def pin_i8_rounding_and_ties(lib):
+    """int8 codes are the nearest integer, ties to even, sign kept; random
+    data equals numpy's round-half-to-even of x / s."""
+    mids = [127.0, 2.5, 3.5, -2.5, -3.5, 0.5, 1.5, -0.5, 126.5, -126.5, -127.0, 0.25]
+    want = [127, 2, 4, -2, -4, 0, 2, 0, 126, -126, -127, 0]
+    codes, scales = oracle.quantize_i8(bf16_bits(mids), 1, lib_path=lib)
+    assert scales[0] == 1.0
+    assert list(codes) == want, list(codes)
+    g = torch.Generator().manual_seed(4)
+    x = (torch.randn(12, 2048, generator=g, dtype=torch.float64)
+         * torch.logspace(-6, 6, 12, base=2.0, dtype=torch.float64)[:, None]).to(torch.bfloat16)
+    x[2, :50] = 0.0
+    codes, scales = oracle.quantize_i8(x, 12, lib_path=lib)
+    ref = np.rint(x.double().numpy() / scales[:, None])
+    np.testing.assert_array_equal(codes.astype(np.float64), ref)
+    deq = oracle.dequantize_i8(codes, scales)
+    assert np.all(np.abs(deq - x.double().numpy()) <= 0.5 * scales[:, None])
+
+
+@pin
+def pin_i8_scale_rule(lib):
+    """Scale = smallest power of two 2^k (k >= -126) with max|x| <= 127 * 2^k:
+    exact boundaries and one bf16 step above them, zeros, tiny and non-finite
+    groups; the largest |code| of a normal group lies in (63, 127]."""
+    for k in (-20, -3, 0, 1, 7, 40):
+        at = 127.0 * 2.0 ** k
+        c, s = oracle.quantize_i8(bf16_bits([at, -1.0 * 2.0 ** k, 0.0, 0.0]), 1, lib_path=lib)
+        assert s[0] == 2.0 ** k and c[0] == 127 and c[1] == -1
+        c, s = oracle.quantize_i8(bf16_bits([0.5 * 2.0 ** k, -128.0 * 2.0 ** k, 0.0, 0.0]), 1, lib_path=lib)
+        assert s[0] == 2.0 ** (k + 1) and c[1] == -64
+    _, s = oracle.quantize_i8(bf16_bits([0.0] * 16), 2, lib_path=lib)
+    assert list(s) == [1.0, 1.0]
+    _, s = oracle.quantize_i8(bf16_bits([2.0 ** -130, 0.0, 0.0, 0.0]), 1, lib_path=lib)
+    assert s[0] == 2.0 ** -126
+    inf16 = torch.tensor([1.0, float("nan"), 2.0, 3.0], dtype=torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    _, s = oracle.quantize_i8(inf16, 2, lib_path=lib)
+    assert np.isnan(s[0]) and s[1] == 2.0 ** -5
+    g = torch.Generator().manual_seed(6)
+    x = (torch.rand(8, 512, generator=g, dtype=torch.float64) * 1000 - 500).to(torch.bfloat16)
+    codes, s = oracle.quantize_i8(x, 8, lib_path=lib)
+    top = np.abs(codes.astype(int)).max(-1)
+    assert np.all((top > 63) & (top <= 127))
+
+
 @pytest.mark.parametrize("fn", PINS, ids=[f.__name__ for f in PINS])
 def test_pin(fn):
     fn(None)

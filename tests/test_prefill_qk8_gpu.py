@@ -1,8 +1,10 @@
-"""GPU parity of the e4m3 quantiser and of the FP8 Q K^T prefill path.
+"""GPU parity of the 8-bit quantisers and of the 8-bit Q K^T prefill paths
+(e4m3 on kind::f8f6f4 MMAs, signed int8 on kind::i8 MMAs).
 
-The quantiser must match the oracle's bit for bit (codes and scales).  The
-prefill with e4m3 Q and K is attention over the dequantised tensors, which
-are exact in bf16 (power-of-two scales, three-bit mantissas): the oracle's
+The quantisers must match the oracle's bit for bit (codes and scales).  The
+prefill with 8-bit Q and K is attention over the dequantised tensors, which
+are exact in bf16 (power-of-two scales, three-bit mantissas or 7-bit
+integers): the oracle's
 own quantisation of the seeded inputs, dequantised, is fed to the fp64
 prefill oracle and the GPU result must meet the usual bar (tolerances and
 skip-mask agreement as in the bf16 prefill tests).  Rule: "Accelerating
@@ -30,15 +32,24 @@ def lib():
     bss.lib()
 
 
-def oracle_dequant_bf16(x, heads=None):
+# format -> (GPU quantiser, GPU prefill, oracle quantiser, oracle dequantiser)
+FORMATS = {
+    "e4m3": (lambda x: bss.quantize_e4m3(x), bss.prefill_qk8, oracle.quantize_e4m3,
+             lambda c, s: oracle.dequantize_e4m3(c, s)),
+    "i8": (lambda x: bss.quantize_i8(x), bss.prefill_qki8, oracle.quantize_i8, oracle.dequantize_i8),
+}
+
+
+def oracle_dequant_bf16(x, heads=None, fmt="e4m3"):
     """The oracle's quantisation of x [B,H,N,d] (optionally of some (b, h)
     slabs only, the rest left as they are), dequantised; exact in bf16."""
+    _, _, oq, odq = FORMATS[fmt]
     B, H, N, d = x.shape
     out = x.clone()
     codes = {}
     for b, h in (heads if heads is not None else [(b, h) for b in range(B) for h in range(H)]):
-        c, s = oracle.quantize_e4m3(x[b, h], 1)
-        deq = oracle.dequantize_e4m3(c, s)
+        c, s = oq(x[b, h], 1)
+        deq = odq(c, s)
         t = torch.from_numpy(deq).to(torch.bfloat16)
         assert np.array_equal(t.double().numpy(), deq), "dequantised value not exact in bf16"
         out[b, h] = t
@@ -46,8 +57,8 @@ def oracle_dequant_bf16(x, heads=None):
     return out, codes
 
 
-def gpu_quant(x):
-    q, s = bss.quantize_e4m3(x.cuda())
+def gpu_quant(x, fmt="e4m3"):
+    q, s = FORMATS[fmt][0](x.cuda())
     torch.cuda.synchronize()
     return q.cpu().numpy(), s.cpu().double().numpy()
 
@@ -58,14 +69,15 @@ def assert_codes_equal(gq, gs, codes):
         np.testing.assert_array_equal(gq[b, h], c)
 
 
-def check(Q, K, V, causal, tau, Bc, units=None, q_heads=None):
-    Q8, qs = bss.quantize_e4m3(Q.cuda())
-    K8, ks = bss.quantize_e4m3(K.cuda())
-    O, mask = bss.prefill_qk8(Q8, K8, qs, ks, V.cuda(), causal, tau, 128, Bc, skip_mask=True)
+def check(Q, K, V, causal, tau, Bc, units=None, q_heads=None, fmt="e4m3"):
+    gq, gp, _, _ = FORMATS[fmt]
+    Q8, qs = gq(Q.cuda())
+    K8, ks = gq(K.cuda())
+    O, mask = gp(Q8, K8, qs, ks, V.cuda(), causal, tau, 128, Bc, skip_mask=True)
     assert bss.attn_sync_status() == 0
     O, mask = O.cpu(), mask.cpu().numpy()
-    Qd, qc = oracle_dequant_bf16(Q, q_heads)
-    Kd, kc = oracle_dequant_bf16(K)
+    Qd, qc = oracle_dequant_bf16(Q, q_heads, fmt)
+    Kd, kc = oracle_dequant_bf16(K, None, fmt)
     assert_codes_equal(Q8.cpu().numpy(), qs.cpu().double().numpy(), qc)
     assert_codes_equal(K8.cpu().numpy(), ks.cpu().double().numpy(), kc)
     r = oracle.prefill(Qd, Kd, V, causal, tau, 128, Bc, units=units, want_exact=False)
@@ -80,16 +92,36 @@ def check(Q, K, V, causal, tau, Bc, units=None, q_heads=None):
 
 
 # ------------------------------------------------------------- quantiser
+@pytest.mark.parametrize("fmt", sorted(FORMATS))
 @pytest.mark.parametrize("shape", [(2, 4, 333, 128), (1, 3, 1, 16), (3, 2, 4096, 64)])
-def test_quantize_matches_oracle_bitwise(shape):
+def test_quantize_matches_oracle_bitwise(shape, fmt):
     B, H, N, d = shape
     g = torch.Generator().manual_seed(N + d)
     x = torch.randn(shape, generator=g, dtype=torch.float64)
     x *= torch.logspace(-20, 20, B * H, base=2.0, dtype=torch.float64).view(B, H, 1, 1)
     x = x.to(torch.bfloat16)
-    gq, gs = gpu_quant(x)
-    _, codes = oracle_dequant_bf16(x)
+    gq, gs = gpu_quant(x, fmt)
+    _, codes = oracle_dequant_bf16(x, None, fmt)
     assert_codes_equal(gq, gs, codes)
+
+
+def test_quantize_i8_special_groups():
+    """int8: a zero head, a head at an exact 127 * 2^k boundary, tiny values,
+    exact ties (2.5 -> 2, 3.5 -> 4, -2.5 -> -2)."""
+    x = torch.zeros(1, 4, 64, 16, dtype=torch.float64)
+    x[0, 1] = torch.linspace(-3, 3, 1024).view(64, 16) * 2.0 ** -4
+    x[0, 1, 0, 0] = 127 * 2.0 ** -4
+    x[0, 2] = torch.linspace(-1, 1, 1024).view(64, 16) * 2.0 ** -125
+    x[0, 3, :, :4] = 2.5
+    x[0, 3, :, 4:8] = 3.5
+    x[0, 3, :, 8:] = -2.5
+    x[0, 3, 0, 0] = 127.0
+    x = x.to(torch.bfloat16)
+    gq, gs = gpu_quant(x, "i8")
+    _, codes = oracle_dequant_bf16(x, None, "i8")
+    assert_codes_equal(gq, gs, codes)
+    assert gs[0, 0] == 1.0 and gs[0, 1] == 2.0 ** -4 and gs[0, 2] == 2.0 ** -126
+    assert (gq[0, 3, 1:, :4] == 2).all() and (gq[0, 3, :, 4:8] == 4).all() and (gq[0, 3, :, 8:] == -2).all()
 
 
 def test_quantize_special_groups():
@@ -121,29 +153,32 @@ def test_quantize_rejects_bad_arguments():
 
 
 # ------------------------------------------------------------- prefill
+@pytest.mark.parametrize("fmt", sorted(FORMATS))
 @pytest.mark.parametrize("Bc", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("N", [300, 512])
-def test_qk8_grid_exact(Bc, causal, N):
+def test_qk8_grid_exact(Bc, causal, N, fmt):
     Q, K, V = inputs.prefill_inputs(2, 4, 2, N, 128, seed=N + Bc + 5, q_sigma=1.5)
-    assert check(Q, K, V, causal, math.inf, Bc) == 0.0
+    assert check(Q, K, V, causal, math.inf, Bc, fmt=fmt) == 0.0
 
 
+@pytest.mark.parametrize("fmt", sorted(FORMATS))
 @pytest.mark.parametrize("Bc", [64, 128])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("tau", [0.0, 2.0, 8.0])
-def test_qk8_grid_skipping(Bc, causal, tau):
+def test_qk8_grid_skipping(Bc, causal, tau, fmt):
     """Inputs with a strong shared direction and sink keys, so many tiles skip."""
     Q, K, V = inputs.prefill_inputs(1, 4, 2, 700, 128, seed=17 + Bc, q_sigma=2.0, q_u=8.0,
                                     sink_scale=6.0)
-    assert check(Q, K, V, causal, tau, Bc) > 0.05
+    assert check(Q, K, V, causal, tau, Bc, fmt=fmt) > 0.05
 
 
+@pytest.mark.parametrize("fmt", sorted(FORMATS))
 @pytest.mark.parametrize("N", [1, 7, 129])
-def test_qk8_tiny_and_ragged(N):
+def test_qk8_tiny_and_ragged(N, fmt):
     Q, K, V = inputs.prefill_inputs(1, 2, 1, N, 128, seed=N)
     for causal in (False, True):
-        check(Q, K, V, causal, 4.0, 128)
+        check(Q, K, V, causal, 4.0, 128, fmt=fmt)
 
 
 def test_qk8_rejects_unsupported():
@@ -159,7 +194,8 @@ def test_qk8_rejects_unsupported():
     assert st == 1
 
 
-def test_qk8_llama3_8b_layer_sampled():
+@pytest.mark.parametrize("fmt", sorted(FORMATS))
+def test_qk8_llama3_8b_layer_sampled(fmt):
     """The 8B causal layer (N = 8192, 32 query / 8 KV heads) at full size,
     checked on sampled row blocks; codes checked on the sampled Q heads and
     every K head."""
@@ -171,4 +207,4 @@ def test_qk8_llama3_8b_layer_sampled():
                    {(0, int(rng.integers(32)), int(rng.integers(n_rb))) for _ in range(6)})
     heads = sorted({(b, h) for b, h, _ in units})
     for tau in (math.inf, 4.0):
-        check(Q, K, V, True, tau, 128, units=units, q_heads=heads)
+        check(Q, K, V, True, tau, 128, units=units, q_heads=heads, fmt=fmt)
