@@ -35,7 +35,7 @@ MUTANTS = {
     "e4m3_subnormal_exponent": ("v = ldexp((double)m, -9);", "v = ldexp((double)m, -10);"),
     "e4m3_scale_not_smallest": ("while (amax > ldexp(448.0, k))", "while (amax >= ldexp(448.0, k))"),
     "e4m3_sign_dropped": ("? 0x80 : 0));", "? 0x00 : 0));"),
-    "i8_ties_away_from_zero": ("(fmod(f, 2.0) == 0.0) ? f : f + 1.0", "f + 1.0"),
+    "i8_ties_upward": ("(fmod(f, 2.0) == 0.0) ? f : f + 1.0", "f + 1.0"),
     "i8_scale_not_smallest": ("while (amax > ldexp(127.0, k))", "while (amax >= ldexp(127.0, k))"),
     "i8_range_128": ("while (amax > ldexp(127.0, k))", "while (amax > ldexp(128.0, k))"),
     "sink_seed_from_second_tile": (
