@@ -426,6 +426,22 @@ def main():
     prefill_extra(MAIN, w, Q, K, V, math.inf, max(3, args.steps // 4), 3)
     prefill_extra(MAIN, w, Q, K, V, 4.0, max(3, args.steps // 4), 2)
     if not args.quick:
+        # the same batch packed as variable-length sequences ([tokens, H, d],
+        # cu_seqlens), the serving layout
+        Qv = Q.permute(0, 2, 1, 3).reshape(-1, w["Hq"], w["d"]).contiguous()
+        Kv = K.permute(0, 2, 1, 3).reshape(-1, w["Hkv"], w["d"]).contiguous()
+        Vv = V.permute(0, 2, 1, 3).reshape(-1, w["Hkv"], w["d"]).contiguous()
+        Ov = torch.empty_like(Qv)
+        cu = torch.arange(0, w["B"] * w["N"] + 1, w["N"], dtype=torch.int32, device=dev)
+        ms_v, _, _ = timed(lambda: bss.prefill_varlen(Qv, Kv, Vv, cu, w["N"], w["causal"], math.inf,
+                                                      w["Br"], w["Bc"], out=Ov),
+                           max(3, args.steps // 4), 2, f"{MAIN} varlen@tau=inf")
+        extras[f"{MAIN} varlen@tau=inf"] = {
+            "ms": ms_v, "dense_tflops": dense_flops(w) / (ms_v * 1e-3) / 1e12,
+            "frac_of_peak": dense_flops(w) / (ms_v * 1e-3) / 1e12 / peaks["bf16_tflops"],
+            "layout": f"{w['B']} sequences of {w['N']} tokens packed as [tokens, H, d]"}
+        del Qv, Kv, Vv, Ov, cu
+    if not args.quick:
         qk8_extra(MAIN, w, Q, K, V, math.inf, max(3, args.steps // 4), 2)
         qk8_extra(MAIN, w, Q, K, V, math.inf, max(3, args.steps // 4), 2, int8=True)
     del Q, K, V, O
@@ -486,6 +502,25 @@ def main():
                     "v_tiles_skipped": 1.0 - v_kept, "row_tiles_skipped": row_skip,
                     "frac_of_hbm": gbs / peaks["hbm_gbs"]}
         decode["rule_variants"] = variants
+        # the same cache as a pool of 64-key pages in shuffled order, read
+        # through a block table (the serving layout)
+        B_, Hkv_, L_, d_ = wd["B"], wd["Hkv"], wd["L"], wd["d"]
+        npg = L_ // 64
+        gen = torch.Generator(device="cpu").manual_seed(7)
+        perm = torch.randperm(B_ * npg, generator=gen).to(dev)
+        Kp = torch.empty(B_ * npg, Hkv_, 64, d_, dtype=torch.bfloat16, device=dev)
+        Vp = torch.empty_like(Kp)
+        Kp[perm] = Kd.view(B_, Hkv_, npg, 64, d_).permute(0, 2, 1, 3, 4).reshape(B_ * npg, Hkv_, 64, d_)
+        Vp[perm] = Vd.view(B_, Hkv_, npg, 64, d_).permute(0, 2, 1, 3, 4).reshape(B_ * npg, Hkv_, 64, d_)
+        table = perm.view(B_, npg).to(torch.int32).contiguous()
+        lens = torch.full((B_,), L_, dtype=torch.int32, device=dev)
+        ms_p, _, _ = timed(lambda: bss.decode_paged(q, Kp, Vp, table, lens, L_, math.inf, out=o),
+                           max(3, args.steps // 4), 2, "decode paged@tau=inf")
+        gbs = 2 * kv_bytes / (ms_p * 1e-3) / 1e9
+        decode["paged@tau=inf"] = {"value": world * gbs, "unit": "GB/s", "latency_us": ms_p * 1000,
+                                   "frac_of_hbm": gbs / peaks["hbm_gbs"],
+                                   "layout": "pool [B*L/64, Hkv, 64, d], pages in a seeded random order"}
+        del Kp, Vp, table, lens, perm
     del q, Kd, Vd, o
     torch.cuda.empty_cache()
 

@@ -241,7 +241,9 @@ __global__ void __launch_bounds__(kPPThreads, 1)
   using C = PPCfg<D, BC, QK8>;
   // variable-length batches store O row by row: a TMA store of the last row
   // block would write into the next sequence's rows
-  constexpr bool kTmaEpi = C::kTmaEpi && !VARLEN;
+  // O by TMA store (variable-length batches: row blocks that end inside
+  // their sequence; the last, partial one of a sequence stores row by row)
+  constexpr bool kTmaEpi = C::kTmaEpi;
   constexpr bool kOSep = C::kOSep && !VARLEN;  // O staged apart from the Q slot
   constexpr int SB = C::kSB;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -843,7 +845,8 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       }
       tc_fence_after();
       const float inv_l = row_valid ? 1.f / l_sum : 0.f;
-      if constexpr (kTmaEpi) {
+      const bool tma_store = kTmaEpi && (!VARLEN || (rb + 1) * kRows <= it.len);
+      if (tma_store) {
         // Stage O (bf16) in this row block's Q tile, which no MMA reads any
         // more (its last S MMA completed before the last P*V), in the TMA
         // layout (64-column panels, 128-byte swizzle), then one thread stores
@@ -873,8 +876,12 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         if (row == 0) {
           release_pending();  // at most one store in flight per warpgroup
 #pragma unroll
-          for (int p = 0; p < C::kVPanels; ++p)
-            tma_store_3d(&tmO, stage + p * C::kQPanel, p * 64, rb * kRows, it.bh);
+          for (int p = 0; p < C::kVPanels; ++p) {
+            if constexpr (VARLEN)  // O as [tokens, Hq, d]
+              tma_store_3d(&tmO, stage + p * C::kQPanel, p * 64, it.bh % Hq, it.tok0 + rb * kRows);
+            else
+              tma_store_3d(&tmO, stage + p * C::kQPanel, p * 64, rb * kRows, it.bh);
+          }
           bulk_commit_group();
           pend_slot = qs;
           pend_n = (t == 0 && it.T1 == 0) ? 2 : 1;  // row block 1 absent: arrive for it too
@@ -897,6 +904,11 @@ __global__ void __launch_bounds__(kPPThreads, 1)
 #pragma unroll
             for (int q = 0; q < 4; ++q) dst[q] = make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
           }
+        }
+        if (kTmaEpi && row == 0) {  // no store reads the Q slot: hand it back like one
+          release_pending();
+          pend_slot = qs;
+          pend_n = (t == 0 && it.T1 == 0) ? 2 : 1;
         }
       }
       // O_t may be overwritten by the next item's first P*V only after this
@@ -1003,7 +1015,7 @@ int pp_launch(const PrefillLaunch& a) {
     if (!pp_map_thd(&mq, a.Q, a.Hq, a.total, D, kRows) ||
         !pp_map_thd(&mk, a.K, a.Hkv, a.total, D, BC) || !pp_map_thd(&mv, a.V, a.Hkv, a.total, D, BC))
       return ATTN_ERR_CUDA;
-    mo = mq;  // unused: variable-length batches store O row by row
+    if (!pp_map_thd(&mo, a.O, a.Hq, a.total, D, kRows)) return ATTN_ERR_CUDA;
     if (a.skip_mask) {  // row blocks past a sequence's end are never visited
       const size_t n = static_cast<size_t>(a.B) * a.Hq * ((a.N + kRows - 1) / kRows) *
                        ((a.N + BC - 1) / BC);

@@ -1,7 +1,7 @@
 """Run one named workload's kernel a few times, for a profiler to capture.
 
     python -m block_skipping_softmax_b200.profile_run --workload llama3_8b_causal_N8192 \
-        --tau inf --launches 3
+        --tau inf --launches 3 [--qk e4m3|i8]
 
 Inputs follow the workload's recipe (drawn on the GPU, as in bench.py); no
 timing is printed, since numbers taken under a profiler are not
@@ -24,6 +24,8 @@ def main(argv=None) -> int:
     ap.add_argument("--workload", required=True, choices=sorted(inputs.WORKLOADS))
     ap.add_argument("--tau", default="inf")
     ap.add_argument("--launches", type=int, default=3)
+    ap.add_argument("--qk", default="bf16", choices=["bf16", "e4m3", "i8"],
+                    help="operand format of Q K^T (prefill; 8-bit inputs are quantised first)")
     args = ap.parse_args(argv)
     tau = math.inf if args.tau == "inf" else float(args.tau)
     w = inputs.WORKLOADS[args.workload]
@@ -32,8 +34,16 @@ def main(argv=None) -> int:
         Q, K, V = inputs.prefill_inputs(w["B"], w["Hq"], w["Hkv"], w["N"], w["d"], seed=0,
                                         device=str(dev), **w["gen"])
         O = torch.empty_like(Q)
-        for _ in range(args.launches):
-            bss.prefill(Q, K, V, w["causal"], tau, w["Br"], w["Bc"], out=O)
+        if args.qk == "bf16":
+            for _ in range(args.launches):
+                bss.prefill(Q, K, V, w["causal"], tau, w["Br"], w["Bc"], out=O)
+        else:
+            quant = bss.quantize_i8 if args.qk == "i8" else bss.quantize_e4m3
+            run = bss.prefill_qki8 if args.qk == "i8" else bss.prefill_qk8
+            Q8, qs = quant(Q)
+            K8, ks = quant(K)
+            for _ in range(args.launches):
+                run(Q8, K8, qs, ks, V, w["causal"], tau, w["Br"], w["Bc"], out=O)
     else:
         q, K, V = inputs.decode_inputs(w["B"], w["Hq"], w["Hkv"], w["L"], w["d"], seed=0, **w["gen"])
         q, K, V = q.to(dev), K.to(dev), V.to(dev)
