@@ -466,14 +466,15 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
         const uint8_t* vt = smem + C::kOffV + vs * C::kTileBytes;
         const float* pr = p_ring + (t % kPRing) * kDecodeTile * G;
         // contiguous cache: rows past L arrive as zeros (with p = 0); paged:
-        // rows past the end of the sequence are whatever the page holds and
-        // are left out
-        const int key_lim_v = PAGED ? Lb - (t_begin + t) * kDecodeTile : kDecodeTile;
+        // rows past the end of the sequence are whatever the page holds (even
+        // NaN), so those keys (p = 0) read the last valid row instead; no
+        // branch, so the loads of all keys issue together
+        const int key_last_v = PAGED ? Lb - (t_begin + t) * kDecodeTile - 1 : kDecodeTile - 1;
 #pragma unroll
         for (int e2 = 0; e2 < C::kVKeys; ++e2) {
           const int key = kg + C::kGroups * e2;
-          if (PAGED && key >= key_lim_v) continue;
-          const uint4 u = *reinterpret_cast<const uint4*>(vt + chunk_off<D>(key, ch));
+          const int key_ld = PAGED ? min(key, key_last_v) : key;
+          const uint4 u = *reinterpret_cast<const uint4*>(vt + chunk_off<D>(key_ld, ch));
           float2 vf[4];
           bf16x8_to_f32(u, vf);
           float pv[G];
