@@ -98,8 +98,8 @@ struct PPCfg {
   static constexpr int kOffO = kOffV + kVS * kVBytes;
   static constexpr int kOffBar = kOffO + (kOSep ? 2 * kOTile : 0);
   // k_full[KS], v_full[VS], commit ring[2][CR], p_full[2][SB], dec[2][DR],
-  // q_full[QS], q_empty[QS], mma_done
-  static constexpr int kNumBars = kKS + kVS + 2 * kCR + 2 * kSB + 2 * kDR + 2 * kQS + 1;
+  // q_full[QS], q_empty[QS], mma_done[2]
+  static constexpr int kNumBars = kKS + kVS + 2 * kCR + 2 * kSB + 2 * kDR + 2 * kQS + 2;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 256 + 1024;
   static constexpr int kTmemCols = 512;
@@ -207,18 +207,22 @@ __device__ __forceinline__ int commits_of(int T) { return T > 0 ? min(SB, T) + T
 // A short FIFO of ring-slot releases: (row block, commit index) that must
 // complete before the slot's next copy.  Fixed positions keep it in registers.
 // The tile number g (running over work items) says when a wait is not needed.
+// A ring slot's last tile: the commit numbers of row blocks 0 and 1 that
+// cover its reads (-1: that row block does not read it), and its running
+// tile number g.
 struct Pending3 {
-  int r[3], c[3], g[3], n;
+  int c0[3], c1[3], g[3], n;
   __device__ __forceinline__ void init() { n = 0; }
-  __device__ __forceinline__ void push(int rr, int cc, int gg) {
-    if (n == 0) { r[0] = rr; c[0] = cc; g[0] = gg; }
-    else if (n == 1) { r[1] = rr; c[1] = cc; g[1] = gg; }
-    else { r[2] = rr; c[2] = cc; g[2] = gg; }
+  // constant indices keep the entries in registers
+  __device__ __forceinline__ void push(int cc0, int cc1, int gg) {
+    if (n == 0) { c0[0] = cc0; c1[0] = cc1; g[0] = gg; }
+    else if (n == 1) { c0[1] = cc0; c1[1] = cc1; g[1] = gg; }
+    else { c0[2] = cc0; c1[2] = cc1; g[2] = gg; }
     ++n;
   }
   __device__ __forceinline__ void pop() {
-    r[0] = r[1]; c[0] = c[1]; g[0] = g[1];
-    r[1] = r[2]; c[1] = c[2]; g[1] = g[2];
+    c0[0] = c0[1]; c1[0] = c1[1]; g[0] = g[1];
+    c0[1] = c0[2]; c1[1] = c1[2]; g[1] = g[2];
     --n;
   }
 };
@@ -265,7 +269,17 @@ __global__ void __launch_bounds__(kPPThreads, 1)
   constexpr int kBQ = kBD + 2 * kDR;
   auto b_q_full = [&](int s) { return bar0 + 8u * (kBQ + s); };
   auto b_q_empty = [&](int s) { return bar0 + 8u * (kBQ + C::kQS + s); };
-  const uint32_t b_mma_done = bar0 + 8u * (kBQ + 2 * C::kQS);
+  // mma_done of MMA issuer 0 and 1 (two issuers at tau = inf)
+  auto b_mma_done = [&](int i) { return bar0 + 8u * (kBQ + 2 * C::kQS + i); };
+  // With tau = inf every V tile is loaded, so tile j of an item is V load
+  // number (tiles of earlier items) + j for both row blocks: each row block
+  // then gets an MMA issuer of its own (warps 1 and 3).  The tcgen05 issue
+  // queue is a few MMAs deep, so a single issuer's waits for one row block
+  // let the pipe run dry while the other row block's work is ready.  With a
+  // finite tau the V loads depend on both row blocks' decisions and warp 1
+  // issues for both.  With one S buffer per row block (Bc = 128 at d = 128)
+  // the single issuer's fixed alternation measured faster, so it stays.
+  const bool dual = tau_is_inf != 0 && SB == 2;
   PPMisc* misc = reinterpret_cast<PPMisc*>(smem + C::kOffMisc);
   volatile int* abort_flag = &misc->abort;
   // keep (1) or skip (0) from the four vote words of one decision
@@ -308,9 +322,11 @@ __global__ void __launch_bounds__(kPPThreads, 1)
     }
     for (int s = 0; s < C::kQS; ++s) {
       mbar_init(b_q_full(s), 1);
-      mbar_init(b_q_empty(s), (kTmaEpi && !kOSep) ? 2 : 1);  // one arrival per row block's O store
+      // one arrival per row block's O store, or per MMA issuer
+      mbar_init(b_q_empty(s), (kTmaEpi && !kOSep) || dual ? 2 : 1);
     }
-    mbar_init(b_mma_done, 1);
+    mbar_init(b_mma_done(0), 1);
+    mbar_init(b_mma_done(1), 1);
     for (int t = 0; t < 2; ++t)
       for (int i = 0; i < kDR; ++i)
         for (int w = 0; w < 4; ++w) misc->vote[t][i][w] = -1;  // no decision number matches
@@ -362,7 +378,8 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         for (int j = 0; j < it.Tmax; ++j) {
           const int s = kload % C::kKS;
           if (pend.n == C::kKS) {  // the slot's previous tile: its S MMAs must have run
-            if (!wait_cm(pend.r[0], pend.c[0])) {
+            if ((pend.c0[0] >= 0 && !wait_cm(0, pend.c0[0])) ||
+                (pend.c1[0] >= 0 && !wait_cm(1, pend.c1[0]))) {
               pp_give_up(misc, status, 2);
               alive = false;
               break;
@@ -378,9 +395,14 @@ __global__ void __launch_bounds__(kPPThreads, 1)
               tma_load_3d(sK + s * C::kKBytes + p * C::kKVPanel, &tmK, b_k_full(s), p * C::kQKCols,
                           j * BC, bkv);
           }
-          // K tile j is read by S of row block 1 last (if it exists, T1 >= T0)
-          if (j < it.T1) pend.push(1, base1 + j, 0);
-          else pend.push(0, base0 + j, 0);
+          // K tile j is read by S_j of each row block that visits it; with
+          // one MMA issuer, row block 1's (if it visits j: T1 >= T0) is last
+          if (dual)
+            pend.push(j < it.T0 ? base0 + j : -1, j < it.T1 ? base1 + j : -1, 0);
+          else if (j < it.T1)
+            pend.push(-1, base1 + j, 0);
+          else
+            pend.push(base0 + j, -1, 0);
           ++kload;
         }
         base0 += commits_of<SB>(it.T0);
@@ -416,7 +438,9 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             // waited for, since their ring slot may have been reused after a
             // run of skipped tiles.
             const bool known_done = !tau_is_inf && pend.g[0] + SB < gbase + j;
-            if (!known_done && !wait_cm(pend.r[0], pend.c[0])) return false;
+            if (!known_done && ((pend.c0[0] >= 0 && !wait_cm(0, pend.c0[0])) ||
+                                (pend.c1[0] >= 0 && !wait_cm(1, pend.c1[0]))))
+              return false;
             pend.pop();
           }
           const int s = vload % C::kVS;
@@ -429,9 +453,15 @@ __global__ void __launch_bounds__(kPPThreads, 1)
               tma_load_3d(sV + s * C::kVBytes + p * C::kKVPanel, &tmV, b_v_full(s), p * 64, j * BC,
                           bkv);
           }
-          // P*V of tile j, row block 1 (if it visits j) is issued after row block 0's
-          if (j < it.T1) pend.push(1, base1 + min(SB, it.T1) + j, gbase + j);
-          else pend.push(0, base0 + min(SB, it.T0) + j, gbase + j);
+          // P*V of tile j by each row block that visits it; with one MMA
+          // issuer, row block 1's (if it visits j) is issued after row block 0's
+          if (dual)
+            pend.push(j < it.T0 ? base0 + min(SB, it.T0) + j : -1,
+                      j < it.T1 ? base1 + min(SB, it.T1) + j : -1, gbase + j);
+          else if (j < it.T1)
+            pend.push(-1, base1 + min(SB, it.T1) + j, gbase + j);
+          else
+            pend.push(base0 + min(SB, it.T0) + j, -1, gbase + j);
           ++vload;
           return true;
         };
@@ -472,8 +502,8 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       }
       for (int t = max(0, vload - C::kVS); t < vload; ++t)
         mbar_drain(b_v_full(t % C::kVS), (t / C::kVS) & 1, wait_limit_ns);
-    } else if (warp == 1 && lane == 0) {
-      // ---------------------------------------------------- MMA issuer
+    } else if ((warp == 1 || (warp == 3 && dual)) && lane == 0) {
+      // ---------------------------------------------------- MMA issuer(s)
       constexpr uint32_t idS = QKT == 2   ? idesc_s8_s32(kRows, BC)
                                : QKT == 1 ? idesc_e4m3_f32(kRows, BC)
                                           : idesc_bf16_f32(kRows, BC, false, false);
@@ -509,6 +539,92 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         mma_commit(b_cm(t, cmc[t]));
         ++cmc[t];
       };
+      const int me = warp == 1 ? 0 : 1;  // the issuer's done barrier (and row block, when dual)
+      if (dual) {
+        // One row block per issuer.  K tile j of an item is K load number
+        // kbase + j (every tile of every item is loaded), and at tau = inf
+        // V tile j is V load number kbase + j as well.  Each row block's
+        // commits keep the single-issuer numbering: min(SB, T) for the
+        // first S tiles, then one per key tile (P*V_j and S_{j+SB}).
+        const int t = me;
+        long long kbase = 0;
+        int pcm = 0, sqm = 0, cmm = 0;  // scalars: a runtime index into the arrays would put them in local memory
+        auto commit_me = [&]() {
+          mma_commit(b_cm(t, cmm));
+          ++cmm;
+        };
+        for (long long k = 0, idx = item_idx(0); alive && idx < n_items; idx = item_idx(++k)) {
+          const Item it = make_item<BC, CAUSAL, VARLEN>(idx, BH, n_pairs, n_rb, N, Hq, cu_seqlens, total);
+          if (VARLEN && it.T0 == 0) continue;  // a pair past the end of its sequence
+          const int T = t == 0 ? it.T0 : it.T1;
+          const int qs = items % C::kQS;
+          ++items;
+          if (T == 0) {  // this row block does not exist: its share of the Q slot release
+            if (!kTmaEpi || kOSep) mbar_arrive(b_q_empty(qs));
+            kbase += it.Tmax;
+            continue;
+          }
+          dQ = sw128_desc_lo(sQ + qs * C::kQSlot, 16);
+          if (!mbar_wait(b_q_full(qs), ((items - 1) / C::kQS) & 1, abort_flag, wait_limit_ns)) {
+            pp_give_up(misc, status, 5);
+            break;
+          }
+          auto wait_k = [&](long long g) -> bool {
+            if (!mbar_wait(b_k_full(static_cast<int>(g % C::kKS)), static_cast<int>(g / C::kKS) & 1,
+                           abort_flag, wait_limit_ns)) {
+              pp_give_up(misc, status, 6);
+              return false;
+            }
+            tc_fence_after();
+            return true;
+          };
+          for (int jj = 0; jj < SB && jj < T; ++jj) {  // S of the first SB key tiles
+            if (!wait_k(kbase + jj)) {
+              alive = false;
+              break;
+            }
+            issue_S(t, static_cast<int>((kbase + jj) % C::kKS), sqm % SB);
+            ++sqm;
+            commit_me();
+          }
+          if (!alive) break;
+          // the Q slot is free once this row block's last S MMA has run
+          if ((!kTmaEpi || kOSep) && T <= SB) mma_commit(b_q_empty(qs));
+          for (int j = 0; alive && j < T; ++j) {
+            const int pb = pcm % SB;
+            if (!mbar_wait(b_p_full(t, pb), (pcm / SB) & 1, abort_flag, wait_limit_ns)) {
+              pp_give_up(misc, status, 7);
+              alive = false;
+              break;
+            }
+            ++pcm;
+            const long long gv = kbase + j;  // V load number of tile j
+            if (!mbar_wait(b_v_full(static_cast<int>(gv % C::kVS)), static_cast<int>(gv / C::kVS) & 1,
+                           abort_flag, wait_limit_ns)) {
+              pp_give_up(misc, status, 8);
+              alive = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t vb = dV0 + static_cast<uint32_t>(gv % C::kVS) * (C::kVBytes >> 4);
+#pragma unroll
+            for (int kk = 0; kk < BC / 16; ++kk)
+              mma_ts(tO(t), tS(t, pb) + kk * 8, desc_join(vb + ((kk * 16 * 128) >> 4), kHi), idPV,
+                     (j > 0 || kk > 0) ? 1u : 0u);
+            if (j + SB < T) {  // S for key tile j + SB reuses the buffer P_t_j just left
+              if (!wait_k(kbase + j + SB)) {
+                alive = false;
+                break;
+              }
+              issue_S(t, static_cast<int>((kbase + j + SB) % C::kKS), sqm % SB);
+              ++sqm;
+            }
+            commit_me();
+            if ((!kTmaEpi || kOSep) && j + SB + 1 == T) mma_commit(b_q_empty(qs));  // last S issued
+          }
+          kbase += it.Tmax;
+        }
+      } else
       for (long long k = 0, idx = item_idx(0); alive && idx < n_items; idx = item_idx(++k)) {
         const Item it = make_item<BC, CAUSAL, VARLEN>(idx, BH, n_pairs, n_rb, N, Hq, cu_seqlens, total);
         if (VARLEN && it.T0 == 0) continue;  // a pair past the end of its sequence
@@ -599,8 +715,8 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         ++items;
       }
       // all issued MMAs must finish before TMEM is released
-      mma_commit(b_mma_done);
-      mbar_drain(b_mma_done, 0, wait_limit_ns);
+      mma_commit(b_mma_done(me));
+      mbar_drain(b_mma_done(me), 0, wait_limit_ns);
     }
   } else {
     reg_inc<C::kSoftmaxRegs>();
