@@ -43,6 +43,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdint>
+#include <type_traits>
 
 #include "kernels.cuh"
 #include "ptx.cuh"
@@ -467,25 +468,32 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
         const float* pr = p_ring + (t % kPRing) * kDecodeTile * G;
         // contiguous cache: rows past L arrive as zeros (with p = 0); paged:
         // rows past the end of the sequence are whatever the page holds (even
-        // NaN), so those keys (p = 0) read the last valid row instead; no
-        // branch, so the loads of all keys issue together
-        const int key_last_v = PAGED ? Lb - (t_begin + t) * kDecodeTile - 1 : kDecodeTile - 1;
+        // NaN), so in a sequence's last, partial tile those keys (p = 0) read
+        // the last valid row instead.  Full tiles take the loop with
+        // compile-time key offsets.
+        auto pv_keys = [&](auto clamp) {
+          const int key_last_v = Lb - (t_begin + t) * kDecodeTile - 1;
 #pragma unroll
-        for (int e2 = 0; e2 < C::kVKeys; ++e2) {
-          const int key = kg + C::kGroups * e2;
-          const int key_ld = PAGED ? min(key, key_last_v) : key;
-          const uint4 u = *reinterpret_cast<const uint4*>(vt + chunk_off<D>(key_ld, ch));
-          float2 vf[4];
-          bf16x8_to_f32(u, vf);
-          float pv[G];
-          load_row_floats<G>(pr + key * G, pv);
+          for (int e2 = 0; e2 < C::kVKeys; ++e2) {
+            const int key = kg + C::kGroups * e2;
+            const int key_ld = decltype(clamp)::value ? min(key, key_last_v) : key;
+            const uint4 u = *reinterpret_cast<const uint4*>(vt + chunk_off<D>(key_ld, ch));
+            float2 vf[4];
+            bf16x8_to_f32(u, vf);
+            float pv[G];
+            load_row_floats<G>(pr + key * G, pv);
 #pragma unroll
-          for (int r = 0; r < G; ++r) {
-            const float2 p2 = make_float2(pv[r], pv[r]);
+            for (int r = 0; r < G; ++r) {
+              const float2 p2 = make_float2(pv[r], pv[r]);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc[r][e] = __ffma2_rn(p2, vf[e], acc[r][e]);
+              for (int e = 0; e < 4; ++e) acc[r][e] = __ffma2_rn(p2, vf[e], acc[r][e]);
+            }
           }
-        }
+        };
+        if (PAGED && Lb - (t_begin + t) * kDecodeTile < kDecodeTile)
+          pv_keys(std::integral_constant<bool, true>{});
+        else
+          pv_keys(std::integral_constant<bool, false>{});
       }
       ++pv_count;
     }
