@@ -9,26 +9,33 @@
 //
 // Layout of one CTA (384 threads, one per SM, persistent):
 //   warpgroup 0: warp 0 TMA Q (both tiles) + K ring; warp 1 TMEM allocator
-//                and the single MMA-issuing thread; warp 2 TMA V ring
-//                (gated by the skip decisions); warp 3 idle.
+//                and an MMA-issuing thread; warp 2 TMA V ring (gated by the
+//                skip decisions); warp 3 the second MMA-issuing thread
+//                (tau = inf with two S buffers per row block: one issuer per
+//                row block), else idle.
 //   warpgroup 1: softmax of row block 0 (thread r owns row r).
 //   warpgroup 2: softmax of row block 1.
 // TMEM (512 columns): O0 | O1 | S/P buffers (two per row block when Bc = 64,
 // one when Bc = 128), P_t (bf16) written over S_t.
 // MMA issue order per key tile j and row block t:  PV_t_j, S_t_{j+SB}, commit
-// so the exponentials of one row block overlap the other block's MMAs.
+// so the exponentials of one row block overlap the other block's MMAs.  The
+// tcgen05 issue queue holds only a few MMAs, so an issuing thread stalls at
+// the pipe's pace; with a single issuer, each of its waits (for one row
+// block's P, or for K or V) lets the pipe run dry, which is why each row
+// block gets its own issuer where the loads allow it.
 //
-// Completion signalling.  A tcgen05.commit stalls the MMA pipe for a few
-// hundred cycles, so the issuer makes exactly one commit per row block and
-// step (plus the first SB S tiles of a work item and one Q-slot release per
-// item), into a ring of mbarriers indexed by a running commit count.  Every
-// completion that a role needs is one of those commits:
+// Completion signalling.  Each issuer makes exactly one commit per row block
+// and step (plus the first SB S tiles of a work item and one Q-slot release
+// per item), into a ring of mbarriers per row block indexed by a running
+// commit count.  Every completion that a role needs is one of those commits:
 //   S_t of key tile i ready         commit #(base_t + i)
 //   P*V_t of key tile j finished    commit #(base_t + min(SB, T_t) + j)
-// (one thread issues every MMA in order, so a commit covers all earlier
-// MMAs).  K and V ring slots, the O rescale and the epilogue all wait on
-// these.  Every wait is bounded; a wait that gives up records a status code
-// and the CTA unwinds (leaving no copy or MMA in flight and freeing TMEM).
+// (a commit covers every earlier MMA of the thread that issues it, and one
+// thread issues all of a row block's MMAs).  K and V ring slots wait for the
+// commits of every row block that reads them; the O rescale and the epilogue
+// wait on their own row block's.  Every wait is bounded; a wait that gives
+// up records a status code and the CTA unwinds (leaving no copy or MMA in
+// flight and freeing TMEM).
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
@@ -548,7 +555,9 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         // first S tiles, then one per key tile (P*V_j and S_{j+SB}).
         const int t = me;
         long long kbase = 0;
-        int pcm = 0, sqm = 0, cmm = 0;  // scalars: a runtime index into the arrays would put them in local memory
+        // scalars: a runtime index into the per-row-block arrays would put
+        // them in local memory
+        int pcm = 0, sqm = 0, cmm = 0;
         auto commit_me = [&]() {
           mma_commit(b_cm(t, cmm));
           ++cmm;
