@@ -54,6 +54,18 @@ def test_status_strings():
 P = 1 << 20  # a 16-byte aligned fake address: validation fails before it is ever used
 
 
+def _cuda_present():
+    import torch
+
+    return torch.cuda.is_available()
+
+
+# Tests that pass fake addresses run only where no GPU can be reached, so a
+# validation gap could never turn into a kernel launch on them.
+no_gpu = pytest.mark.skipif(_cuda_present(), reason="fake device addresses are passed only without a GPU")
+
+
+@no_gpu
 @pytest.mark.parametrize("args", [
     dict(Q=0), dict(O=0), dict(B=0), dict(N=-1), dict(Hq=3, Hkv=2), dict(d=96),
     dict(Br=64, Bc=128), dict(Br=32, Bc=32), dict(tau=float("nan")), dict(tau=-1.0),
@@ -67,6 +79,7 @@ def test_prefill_rejects_bad_arguments(args):
     assert st == 1
 
 
+@no_gpu
 @pytest.mark.parametrize("args", [
     dict(q=0), dict(L=0), dict(Hq=4, Hkv=3), dict(d=32), dict(tau=float("nan")), dict(tau=-0.5),
     dict(K=P + 4),
@@ -78,6 +91,7 @@ def test_decode_rejects_bad_arguments(args):
     assert st == 1
 
 
+@no_gpu
 def test_decode_rejects_bad_workspace():
     st = bss.attn_decode_ex(P, P, P, P, 1, 4, 1, 1000, 128, 1.0, None, None, None, 64)
     assert st == 1
@@ -102,3 +116,62 @@ def test_split_len_is_deterministic_and_tiles_the_keys():
 def test_wait_limit_validation():
     assert bss.attn_set_wait_limit_ms(0) == 1
     assert bss.attn_set_wait_limit_ms(2000) == 0
+
+
+@no_gpu
+@pytest.mark.parametrize("fn", ["attn_quantize_e4m3", "attn_quantize_i8"])
+@pytest.mark.parametrize("args", [
+    dict(x=0), dict(q=0), dict(scales=0), dict(groups=0), dict(group_elems=0), dict(group_elems=24),
+    dict(x=P + 8), dict(q=P + 4), dict(scales=P + 2),
+])
+def test_quantize_rejects_bad_arguments(fn, args):
+    a = dict(x=P, q=P, scales=P, groups=4, group_elems=1024)
+    a.update(args)
+    st = getattr(bss, fn)(a["x"], a["q"], a["scales"], a["groups"], a["group_elems"])
+    assert st == 1
+
+
+@no_gpu
+@pytest.mark.parametrize("fn", ["attn_prefill_qk8", "attn_prefill_qki8"])
+@pytest.mark.parametrize("args", [
+    dict(qs=0), dict(ks=0), dict(qs=P + 2), dict(d=64), dict(Br=64, Bc=64), dict(Q8=0), dict(V=P + 8),
+    dict(tau=float("nan")), dict(Hq=3, Hkv=2),
+])
+def test_prefill_8bit_rejects_bad_arguments(fn, args):
+    a = dict(Q8=P, K8=P, qs=P, ks=P, V=P, O=P, B=1, Hq=2, Hkv=1, N=256, d=128, causal=1, tau=1.0,
+             Br=128, Bc=128)
+    a.update(args)
+    st = getattr(bss, fn)(a["Q8"], a["K8"], a["qs"], a["ks"], a["V"], a["O"], a["B"], a["Hq"], a["Hkv"],
+                          a["N"], a["d"], a["causal"], a["tau"], a["Br"], a["Bc"])
+    assert st == 1
+
+
+@no_gpu
+@pytest.mark.parametrize("args", [
+    dict(cu=0), dict(cu=P + 2), dict(total=0), dict(maxlen=0), dict(Br=64, Bc=64), dict(d=96),
+])
+def test_prefill_varlen_rejects_bad_arguments(args):
+    a = dict(Q=P, K=P, V=P, O=P, cu=P, B=2, maxlen=300, total=500, Hq=2, Hkv=1, d=128, causal=1,
+             tau=1.0, Br=128, Bc=64)
+    a.update(args)
+    st = bss.attn_prefill_varlen(a["Q"], a["K"], a["V"], a["O"], a["cu"], a["B"], a["maxlen"], a["total"],
+                                 a["Hq"], a["Hkv"], a["d"], a["causal"], a["tau"], a["Br"], a["Bc"])
+    assert st == 1
+
+
+def test_python_wrappers_reject_host_tensors():
+    """The marshalling layer refuses tensors that are not CUDA tensors of the
+    expected type before it reaches the library (there is no CPU path)."""
+    import torch
+
+    x = torch.zeros(1, 1, 128, 128, dtype=torch.bfloat16)
+    with pytest.raises(bss.AttnError):
+        bss.quantize_e4m3(x)
+    with pytest.raises(bss.AttnError):
+        bss.quantize_i8(x)
+    q8 = torch.zeros(1, 1, 128, 128, dtype=torch.uint8)
+    s = torch.ones(1, 1)
+    with pytest.raises(bss.AttnError):
+        bss.prefill_qk8(q8, q8, s, s, x, True)
+    with pytest.raises(bss.AttnError):
+        bss.prefill(x, x, x, True)
