@@ -26,6 +26,8 @@ def main(argv=None) -> int:
     ap.add_argument("--launches", type=int, default=3)
     ap.add_argument("--qk", default="bf16", choices=["bf16", "e4m3", "i8"],
                     help="operand format of Q K^T (prefill; 8-bit inputs are quantised first)")
+    ap.add_argument("--paged", action="store_true",
+                    help="decode: read the cache as a pool of 64-key pages in seeded random order")
     args = ap.parse_args(argv)
     tau = math.inf if args.tau == "inf" else float(args.tau)
     w = inputs.WORKLOADS[args.workload]
@@ -48,8 +50,23 @@ def main(argv=None) -> int:
         q, K, V = inputs.decode_inputs(w["B"], w["Hq"], w["Hkv"], w["L"], w["d"], seed=0, **w["gen"])
         q, K, V = q.to(dev), K.to(dev), V.to(dev)
         o = torch.empty_like(q)
-        for _ in range(args.launches):
-            bss.decode(q, K, V, tau, out=o)
+        if args.paged:
+            B, Hkv, L, d = w["B"], w["Hkv"], w["L"], w["d"]
+            npg = -(-L // 64)
+            assert L % 64 == 0, "the page pool here holds whole pages"
+            perm = torch.randperm(B * npg, generator=torch.Generator().manual_seed(7)).to(dev)
+            Kp = torch.empty(B * npg, Hkv, 64, d, dtype=torch.bfloat16, device=dev)
+            Vp = torch.empty_like(Kp)
+            Kp[perm] = K.view(B, Hkv, npg, 64, d).permute(0, 2, 1, 3, 4).reshape(B * npg, Hkv, 64, d)
+            Vp[perm] = V.view(B, Hkv, npg, 64, d).permute(0, 2, 1, 3, 4).reshape(B * npg, Hkv, 64, d)
+            table = perm.view(B, npg).to(torch.int32).contiguous()
+            lens = torch.full((B,), L, dtype=torch.int32, device=dev)
+            del K, V
+            for _ in range(args.launches):
+                bss.decode_paged(q, Kp, Vp, table, lens, L, tau, out=o)
+        else:
+            for _ in range(args.launches):
+                bss.decode(q, K, V, tau, out=o)
     st = bss.attn_sync_status()
     if st != 0:
         print(f"kernel status {bss.attn_status_string(st)}", file=sys.stderr)
