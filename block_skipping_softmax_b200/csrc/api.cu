@@ -100,6 +100,11 @@ void host_pipeline_release();  // host_pipeline.cu
 // points defined in other files.
 int device_context(int* dev, int** status) { return device_ready(dev, status); }
 unsigned long long wait_limit_ns() { return g_wait_limit_ns; }
+// The decode argument checks, for decode entry points defined in other files.
+int check_decode_args(const void* q, const void* K, const void* V, const void* o, int B, int Hq,
+                      int Hkv, int L, int d, float tau) {
+  return check_decode(q, K, V, o, B, Hq, Hkv, L, d, tau);
+}
 }  // namespace bss
 
 extern "C" {

@@ -26,6 +26,8 @@
 namespace bss {
 int device_context(int* dev, int** status);  // defined in api.cu
 unsigned long long wait_limit_ns();          // defined in api.cu
+int check_decode_args(const void* q, const void* K, const void* V, const void* o, int B, int Hq,
+                      int Hkv, int L, int d, float tau);  // defined in api.cu
 }
 
 namespace {
@@ -59,16 +61,9 @@ int scratch_address(int dev, void** out) {
 extern "C" int attn_decode_noalloc(const void* q, const void* K, const void* V, void* o, int B,
                                    int Hq, int Hkv, int L, int d, float tau, void* stream,
                                    uint8_t* skip_mask) {
-  if (!q || !K || !V || !o) return ATTN_ERR_INVALID_ARG;
-  const uintptr_t mis = (reinterpret_cast<uintptr_t>(q) | reinterpret_cast<uintptr_t>(K) |
-                         reinterpret_cast<uintptr_t>(V) | reinterpret_cast<uintptr_t>(o)) & 15u;
-  if (mis) return ATTN_ERR_INVALID_ARG;
-  if (B <= 0 || Hq <= 0 || Hkv <= 0 || L <= 0 || Hq % Hkv != 0) return ATTN_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return ATTN_ERR_INVALID_ARG;
-  if (std::isnan(tau) || tau < 0.f) return ATTN_ERR_INVALID_ARG;
-  const int g = Hq / Hkv;
-  if (g != 1 && g != 2 && g != 4 && g != 8) return ATTN_ERR_UNSUPPORTED;
-  if (Hkv > 65535 || B > 65535) return ATTN_ERR_UNSUPPORTED;
+  // the same argument checks as attn_decode_ex, before any CUDA call
+  int st = bss::check_decode_args(q, K, V, o, B, Hq, Hkv, L, d, tau);
+  if (st != ATTN_OK) return st;
 
   // same split layout as attn_decode, so results are identical
   const int ls = attn_decode_split_len(B, Hkv, L);
@@ -79,13 +74,14 @@ extern "C" int attn_decode_noalloc(const void* q, const void* K, const void* V, 
 
   int dev = 0;
   int* status = nullptr;
-  int st = bss::device_context(&dev, &status);
+  st = bss::device_context(&dev, &status);
   if (st != ATTN_OK) return st;
   void* scratch = nullptr;
   if ((st = scratch_address(dev, &scratch)) != ATTN_OK) return st;
 
   // Every scratch entry the combine kernel reads is written earlier in the
-  // same call by the partial kernel, so nothing needs clearing.
+  // same call by the partial kernel (a CTA whose bounded wait gives up writes
+  // its split as empty), so nothing needs clearing.
   bss::DecodeLaunch a{};
   a.q = q;
   a.K = K;

@@ -513,6 +513,13 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
           mbar_drain(b_v_full(k % kVStages), (k / kVStages) & 1, wait_limit_ns);
       if (seed_issued) mbar_drain(b_seed, 0, wait_limit_ns);
     }
+    // this split's partials are written as an empty split (zero weight in the
+    // merge), so the output never mixes in scratch left by an earlier call
+    for (int idx = tid; idx < G * D; idx += kDecThreads) {
+      const size_t row = static_cast<size_t>(b) * Hq + kv * G + idx / D;
+      o_part[(row * n_splits + split) * D + idx % D] = 0.f;
+    }
+    if (tid < G) lse_part[(static_cast<size_t>(b) * Hq + kv * G + tid) * n_splits + split] = NEG_INF;
     return;
   }
 
@@ -591,7 +598,8 @@ __global__ void __launch_bounds__(D)
     den += w;
     num = fmaf(w, o_part[(static_cast<size_t>(row) * n_splits + s) * D + col], num);
   }
-  o[static_cast<size_t>(row) * D + col] = __float2bfloat16_rn(num / den);
+  // every split empty (only after a wait gave up): 0 rather than NaN
+  o[static_cast<size_t>(row) * D + col] = __float2bfloat16_rn(den > 0.f ? num / den : 0.f);
 }
 
 namespace {

@@ -883,8 +883,10 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           m_ref = m_cand;
         }
         // P = 2^(s*scale - m_ref): one packed FFMA per pair, two ex2, one
-        // pack to bf16 for the P*V MMA; the row sum adds the fp32 pair with
-        // one packed add (four independent chains)
+        // pack to bf16 for the P*V MMA.  The row sum adds the bf16-rounded
+        // pair that the P*V MMA multiplies (one packed add, four independent
+        // chains), so numerator and denominator see the same weights and the
+        // rounding of a dominant weight cancels in O / l.
         // invalid rows: all scores -inf -> P = 0; int8 scores carry the
         // offset 1.5 * 2^23, taken out here
         const float neg_m = (row_valid ? -m_ref : 0.f) - (QKT == 2 ? kI2FOffset * sl2 : 0.f);
@@ -901,16 +903,10 @@ __global__ void __launch_bounds__(kPPThreads, 1)
                 make_float2(__uint_as_float(u[c0 + 2 * c]), __uint_as_float(u[c0 + 2 * c + 1])), sc2,
                 nm2);
             // pairs in kPolyPairs take 2^x on the FMA pipes, the rest on MUFU
-            uint32_t w;
-            if ((kPolyPairs >> c) & 1u) {  // 2^x on the FMA pipes; the sum takes the bf16 values
-              w = exp2_poly_bf16x2(x);
-              rs2[c & 3] = __fadd2_rn(rs2[c & 3], make_float2(__uint_as_float(w << 16),
-                                                              __uint_as_float(w & 0xffff0000u)));
-            } else {  // 2^x on MUFU; the sum takes the fp32 values
-              const float2 e = make_float2(ex2(x.x), ex2(x.y));
-              w = pack_bf16x2(e.x, e.y);
-              rs2[c & 3] = __fadd2_rn(rs2[c & 3], e);
-            }
+            const uint32_t w = ((kPolyPairs >> c) & 1u) ? exp2_poly_bf16x2(x)
+                                                        : pack_bf16x2(ex2(x.x), ex2(x.y));
+            rs2[c & 3] = __fadd2_rn(rs2[c & 3], make_float2(__uint_as_float(w << 16),
+                                                            __uint_as_float(w & 0xffff0000u)));
             pk[c] = w;
           }
           tmem_st16(tS(t, sb) + lane_off + c0 / 2, pk);

@@ -1,9 +1,9 @@
-// 8-bit quantisation of Q or K for the low-precision Q K^T prefill paths
-// ("Accelerating Long-Context Inference with Skip Softmax in NVIDIA
-// TensorRT-LLM": the skip test runs on the raw Q K^T scores, which may come
-// from lower-precision operands; the page names FP8 attention as the path it
-// combines with; "TurboAttention", Technical Deep Dive: integer Q K^T inside
-// the tile loop).
+// 8-bit quantisation of Q or K for the low-precision Q K^T prefill paths.
+// The int8 path follows "TurboAttention: Efficient Attention Approximation
+// for High-Throughput LLM Serving" (Technical Deep Dive), which quantises Q
+// and K to integers inside the FlashAttention tile loop.  No page names FP8:
+// the e4m3 path is this library's own choice of a second 8-bit format on the
+// same pipeline (the B200 tensor cores run e4m3 at the int8 rate).
 //
 // A tensor is cut into `groups` contiguous groups (one head slab [N, d] each
 // for the prefill layouts).  Each group gets one power-of-two scale s, the

@@ -29,6 +29,11 @@
  *     attn_sync_status().
  *   - There is no CPU fallback: without an sm_100 device every compute call
  *     returns ATTN_ERR_UNSUPPORTED.
+ *   - The library caches, per device ordinal, the device addresses of its
+ *     own __device__ variables (the status word, the no-alloc scratch) in
+ *     the device's primary context.  Use it only from the primary context
+ *     (the CUDA runtime's default), and not across cudaDeviceReset: after a
+ *     reset the cached addresses would be stale.
  */
 #ifndef SKIP_SOFTMAX_ATTN_H
 #define SKIP_SOFTMAX_ATTN_H
@@ -272,8 +277,10 @@ ATTN_API int attn_decode_paged(const void* q, const void* K_pages, const void* V
  *   The first call on a device looks up that array's device address; make
  *   that first call before any stream capture.  Every call shares the array
  *   and leaves its contents behind (nothing in it needs clearing: each entry
- *   read is written earlier in the same call), so calls that overlap on the
- *   GPU -- on different streams, or from different threads -- race.
+ *   read is written earlier in the same call, also when a bounded wait gives
+ *   up, in which case o is 0 for the affected rows and attn_sync_status()
+ *   reports ATTN_ERR_TIMEOUT), so calls that overlap on the GPU -- on
+ *   different streams, or from different threads -- race.
  *   Errors: as attn_decode_ex, plus ATTN_ERR_UNSUPPORTED when the problem
  *   needs more than 16 MiB of scratch (about B*Hq*splits*(d+1)*4 bytes).
  *   Calls no cudaMalloc, cudaFree or allocating library routine.

@@ -4,26 +4,25 @@ Bar (fixed for this method): bf16 outputs within max-abs 1e-2 and mean-abs
 1e-3 of the fp64 oracle (fp32 accumulation on the GPU); skip masks identical
 except tiles whose oracle margin lies within 1e-3 of the threshold.
 
-Where a reference output has |O| >= 2, the spacing of the bf16 grid (one ulp,
-2^-6 = 0.0156 and up) is wider than 1e-2: the correctly rounded value alone
-may sit 0.0078 away, and any upstream error of a few 1e-3 (the bf16 rounding
-of the probabilities that feed the P*V product is 2^-8 relative) moves the
-result to the neighbouring grid point.  Such elements must lie within one
-bf16 ulp of the exact value instead; their count is returned.
+Where a reference output has |O| >= 4, half the spacing of the bf16 grid
+(2^-6 = 0.0156 and up) is already wider than 1e-2: the correctly rounded
+value alone may sit that far away.  Only there may an element differ from
+the exact value by up to one bf16 ulp instead of 1e-2.  Everywhere else
+(|O| < 4) the 1e-2 bound holds without exception; the count of elements
+that used the one-ulp allowance is printed and returned.
 """
-import math
-
 import numpy as np
 import torch
 
 MAX_ABS = 1e-2
 MEAN_ABS = 1e-3
 MARGIN_BAND = 1e-3
+ULP_BAND = 4.0  # |O| from which the bf16 half-ulp exceeds MAX_ABS
 
 
 def _elem_tol(ref):
     ulp = np.exp2(np.floor(np.log2(np.maximum(np.abs(ref), 1e-30))) - 7)  # one bf16 ulp
-    return np.maximum(MAX_ABS, np.where(np.abs(ref) >= 2, ulp, 0.0))
+    return np.maximum(MAX_ABS, np.where(np.abs(ref) >= ULP_BAND, ulp, 0.0))
 
 
 def compare_masks(gpu_mask, ref_mask, ref_margin):
@@ -44,12 +43,17 @@ def compare_outputs(gpu, ref, rows_mask=None, what="O"):
         sel &= rows_mask
     assert sel.any(), "nothing to compare"
     err = np.abs(g - ref)[sel]
+    aref = np.abs(ref)[sel]
     tol = _elem_tol(ref)[sel]
     worst = float(err.max())
     mean = float(err.mean())
+    # below the one-ulp band the plain bound holds for every element
+    n_over_small = int(((err > MAX_ABS) & (aref < ULP_BAND)).sum())
+    assert n_over_small == 0, f"{what}: {n_over_small} elements with |O| < {ULP_BAND} off by > {MAX_ABS}"
     assert np.all(err <= tol), f"{what}: max abs error {worst:.3g} above tolerance"
     assert mean <= MEAN_ABS, f"{what}: mean abs error {mean:.3g} > {MEAN_ABS}"
-    n_wide = int((err > MAX_ABS).sum())  # elements that needed the one-ulp allowance
+    n_wide = int((err > MAX_ABS).sum())  # elements (all with |O| >= 4) that used the one-ulp allowance
+    print(f"[parity] {what}: max {worst:.3g} mean {mean:.3g} n={err.size} one-ulp-allowance={n_wide}")
     return worst, mean, n_wide
 
 

@@ -84,11 +84,30 @@ def test_prefill_rejects_bad_arguments(args):
     dict(q=0), dict(L=0), dict(Hq=4, Hkv=3), dict(d=32), dict(tau=float("nan")), dict(tau=-0.5),
     dict(K=P + 4),
 ])
-def test_decode_rejects_bad_arguments(args):
+@pytest.mark.parametrize("entry", ["attn_decode", "attn_decode_noalloc"])
+def test_decode_rejects_bad_arguments(args, entry):
     a = dict(q=P, K=P, V=P, o=P, B=1, Hq=4, Hkv=1, L=1000, d=128, tau=2.0)
     a.update(args)
-    st = bss.attn_decode(a["q"], a["K"], a["V"], a["o"], a["B"], a["Hq"], a["Hkv"], a["L"], a["d"], a["tau"])
+    pos = (a["q"], a["K"], a["V"], a["o"], a["B"], a["Hq"], a["Hkv"], a["L"], a["d"], a["tau"])
+    if entry == "attn_decode":
+        st = bss.attn_decode(*pos)
+    else:
+        st = bss.attn_decode_noalloc(*pos, None, None)
     assert st == 1
+
+
+@no_gpu
+def test_decode_noalloc_rejects_problems_beyond_its_array():
+    """The no-alloc decode refuses a problem whose split scratch exceeds its
+    fixed 16 MiB array, before any CUDA call (so no GPU is needed to test it)."""
+    B, Hq, Hkv, L, d = 512, 64, 8, 64, 128
+    ls = bss.attn_decode_split_len(B, Hkv, L)
+    n_splits = -(-L // ls)
+    r256 = lambda x: (x + 255) // 256 * 256
+    need = r256(B * Hq * n_splits * d * 4) + r256(B * Hq * n_splits * 4)
+    assert need > 16 << 20, "shape must exceed the no-alloc scratch array"
+    st = bss.attn_decode_noalloc(P, P, P, P, B, Hq, Hkv, L, d, 1.0, None, None)
+    assert st == 2, bss.attn_status_string(st)
 
 
 @no_gpu

@@ -15,7 +15,6 @@ import torch
 import block_skipping_softmax_b200 as bss
 from block_skipping_softmax_b200 import build as bss_build
 from block_skipping_softmax_b200 import inputs
-from parity import compare_masks, compare_outputs
 
 pytestmark = pytest.mark.gpu
 
@@ -61,27 +60,5 @@ def test_no_alloc_matches_regular_entry_point_twice():
         torch.cuda.synchronize()
         assert bss.attn_sync_status() == 0
         np.testing.assert_array_equal(m_new.cpu().numpy(), m_ref.cpu().numpy())
-        compare_outputs(o_new.cpu(), o_ref.float().cpu().double().numpy(), what="o (no-alloc)")
-
-
-def test_no_alloc_rejects_problems_beyond_its_array():
-    """A problem whose split scratch exceeds the fixed 16 MiB array is refused.
-
-    The buffers are real and sized for the problem, and the test first checks
-    from the split layout that the scratch really exceeds the array, so the
-    call cannot reach a kernel with memory it does not own."""
-    B, Hq, Hkv, L, d = 512, 64, 8, 64, 128
-    ls = bss.attn_decode_split_len(B, Hkv, L)
-    n_splits = -(-L // ls)
-    r256 = lambda x: (x + 255) // 256 * 256
-    need = r256(B * Hq * n_splits * d * 4) + r256(B * Hq * n_splits * 4)
-    assert need > 16 << 20, "shape must exceed the no-alloc scratch array"
-    q = torch.zeros(B, Hq, d, dtype=torch.bfloat16, device="cuda")
-    K = torch.zeros(B, Hkv, L, d, dtype=torch.bfloat16, device="cuda")
-    V = torch.zeros_like(K)
-    o = torch.empty_like(q)
-    st = bss.attn_decode_noalloc(q.data_ptr(), K.data_ptr(), V.data_ptr(), o.data_ptr(), B, Hq, Hkv, L,
-                                 d, 1.0, torch.cuda.current_stream().cuda_stream, None)
-    assert st == 2, bss.attn_status_string(st)
-    torch.cuda.synchronize()
-    assert bss.attn_sync_status() == 0
+        # the same kernels over the same split layout: bit-identical outputs
+        assert torch.equal(o_new, o_ref), "no-alloc decode differs from attn_decode_ex"
