@@ -1,25 +1,34 @@
 """Benchmark of Skip Softmax attention on B200 (prefill and decode).
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl own|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl own|reference] [--quick]
 
-One JSON line on stdout (rank 0).  Headline (``value``): prefill
-dense-equivalent TFLOP/s on the non-causal encoder workload
-(B=64, Hq=Hkv=32, N=512, d=128, Br=128, Bc=64, tau=inf) -- a step is one
-attn_prefill call over that batch, inputs resident in HBM.  The decode half
-of the metric (KV-read GB/s on B=16, Hq=32, Hkv=8, L=32768, d=128) is timed
-the same way and reported under ``decode``; the other workloads and
-thresholds are under ``workloads``.
+One JSON line on stdout (rank 0).
 
-Timing: W untimed warm-up steps, then exactly K steps between two CUDA events
-on the launching stream, bracketed by a barrier and a device synchronise, max
-over ranks.  Every workload's inputs (>= 1.07 GB, or 168 MB for the 8B layer)
-are larger than the 126 MB L2, so consecutive steps do not hit in L2.
-Multi-GPU: every rank runs its own copy of the workload (independent
-sequences; no collective on the data path) -> weak scaling.
+Headline (``value``): prefill dense-equivalent TFLOP/s on the causal
+Llama-3.3-70B attention-layer shape at 128K context (B=1, Hq=64, Hkv=8,
+N=131072, d=128, Br=Bc=128, tau=inf), the largest workload and the one the
+Skip Softmax page reports on.  A step is one attn_prefill call over that
+layer, inputs resident in HBM.
+
+``configs`` holds one entry per workload (the five shapes of
+``inputs.WORKLOADS``) at each of its thresholds: prefill dense-equivalent and
+executed TFLOP/s, the skipped fraction, latency and the fraction of the
+measured bf16 peak; decode KV-read GB/s, latency and the fraction of the
+measured HBM bandwidth.  ``extras`` holds the rest (8-bit Q K^T, varlen,
+decode rule variants, paged decode, and an input on which the skip rule
+fires), none of which is one of the five workloads.
+
+Timing: W untimed warm-up steps (at least 3), then exactly K steps between
+two CUDA events on the launching stream, bracketed by a barrier and a device
+synchronise, max over ranks.  Every timed workload but the 256-token one has
+inputs larger than the 126 MB L2 (the 8B layer: 168 MB); the 256-token one
+fits in L2 by construction and is launch-bound.  Multi-GPU: every rank runs
+its own copy of the workload (independent sequences; no collective on the
+data path) -> weak scaling.
 
 ``--impl reference`` times the fp64 CPU oracle (the deliberately slow
-reference program) on a bounded sample of the same workload, on this host's
-cores, in the same unit.
+reference program) on a bounded sample of the headline workload, on this
+host's cores, in the same unit.
 """
 from __future__ import annotations
 
@@ -37,10 +46,22 @@ import time
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-MAIN = "encoder_64x32x512_d128"
+HEADLINE = "llama33_70b_causal_N131072"
+ENCODER = "encoder_64x32x512_d128"
 DECODE = "gqa_decode_16x32q8kv_L32768"
+LAYER_8B = "llama3_8b_causal_N8192"
+SMALL = "causal_1x1x256_d64"
+CONFIG_ORDER = [SMALL, ENCODER, DECODE, LAYER_8B, HEADLINE]
 METRIC = "prefill attn TFLOP/s (dense-equiv) & % tensor peak; decode KV-read GB/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+PAGES_CONTEXT = {
+    "source": "Accelerating Long-Context Inference with Skip Softmax in NVIDIA TensorRT-LLM "
+              "(Key Points; Detailed Analysis)",
+    "decode_end_to_end_speedup": "about 1.4x, Llama 3.3 70B, NVIDIA GB200 system",
+    "prefill_speedup": "about 40% at 128K context, Llama 3.3 70B, NVIDIA GB200 system",
+    "turboattention_profiling_hardware": "NVIDIA A100 (TurboAttention: Efficient Attention "
+                                         "Approximation for High-Throughput LLM Serving)",
+}
 
 
 def load_peaks():
@@ -53,9 +74,10 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
-def measured_traffic(kernel: str, cu_file: str):
-    """DRAM bytes per launch from the committed ncu summary, or None when the
-    kernel's source changed since the counters were taken."""
+def measured_traffic(key: str, cu_file: str):
+    """DRAM bytes per launch from the committed ncu record, or None when the
+    kernel's source changed since the counters were taken.  ``key`` names the
+    kernel and the workload the counters were taken on."""
     import hashlib
 
     csrc = os.path.join(ROOT, "block_skipping_softmax_b200", "csrc")
@@ -68,7 +90,7 @@ def measured_traffic(kernel: str, cu_file: str):
         with open(os.path.join(ROOT, "profiles", "ncu_traffic.txt")) as fh:
             for line in fh:
                 parts = line.split()
-                if len(parts) >= 3 and not line.startswith("#") and parts[0] == kernel and parts[1] == digest:
+                if len(parts) >= 3 and not line.startswith("#") and parts[0] == key and parts[1] == digest:
                     return int(parts[2])
     except OSError:
         pass
@@ -84,6 +106,13 @@ def compulsory_prefill_bytes(w):
     return 2 * w["B"] * w["Hq"] * w["N"] * w["d"] * 2 + 2 * w["B"] * w["Hkv"] * w["N"] * w["d"] * 2
 
 
+def headline_config(w, world):
+    return {"workload": HEADLINE, "B": w["B"], "Hq": w["Hq"], "Hkv": w["Hkv"], "N": w["N"], "d": w["d"],
+            "causal": w["causal"], "Br": w["Br"], "Bc": w["Bc"], "tau": "inf",
+            "parallelism": f"replicas x{world} (independent sequences)",
+            "l2": "inputs 4.83 GB per step > 126 MB L2 (no flush needed)"}
+
+
 class ClockSampler:
     """nvidia-smi clocks and throttle reasons, sampled every 100 ms."""
 
@@ -95,7 +124,6 @@ class ClockSampler:
         self.rows = []
         self.proc = None
         self.gpu = gpu_index
-        self.t_start = None
 
     def start(self):
         try:
@@ -111,9 +139,6 @@ class ClockSampler:
     def _read(self):
         for line in self.proc.stdout:
             self.rows.append((time.time(), [x.strip() for x in line.split(",")]))
-
-    def mark(self):
-        return time.time()
 
     def stop(self):
         if self.proc is not None:
@@ -157,49 +182,61 @@ def cpu_cores():
 
 
 # --------------------------------------------------------------------------- CPU oracle
-def oracle_sample_rate(w, target_s, Q=None, K=None, V=None, seed=1):
-    """Time the fp64 oracle on a sample of row blocks of workload w (~target_s
-    of CPU work).  Returns (TFLOP/s, seconds, n_row_blocks, cores)."""
+_ORACLE_INPUTS = {}
+
+
+def oracle_sample_headline(target_s, seed=1, heads=None, n_units=None):
+    """Time the fp64 oracle on a random sample of row blocks of the headline
+    workload (~target_s of CPU work on all host cores).
+
+    The row blocks come from a few query heads, each drawn on its own with its
+    KV head (bit for bit the heads of the full layer) and stacked as a small
+    batch of independent heads, since the oracle's output buffers for all 64
+    heads of a 128K-token layer would not fit in host memory.  ``n_units``
+    fixes the sample size (row blocks per call); otherwise a short calibration
+    run sizes it to ``target_s``.  Returns (TFLOP/s, seconds, row blocks,
+    cores, heads)."""
     import numpy as np
+    import torch
 
     import oracle
     from block_skipping_softmax_b200 import inputs
 
-    if Q is None:
-        Q, K, V = inputs.prefill_inputs(w["B"], w["Hq"], w["Hkv"], w["N"], w["d"], seed=0, **w["gen"])
-    n_rb = -(-w["N"] // w["Br"])
+    w = inputs.WORKLOADS[HEADLINE]
     rng = np.random.default_rng(seed)
-    all_units = [(b, h, rb) for b in range(w["B"]) for h in range(w["Hq"]) for rb in range(n_rb)]
+    if heads is None:
+        heads = sorted(int(h) for h in rng.choice(w["Hq"], 4, replace=False))
+    key = tuple(heads)
+    if key not in _ORACLE_INPUTS:  # drawn once per set of heads
+        drawn = [inputs.prefill_head_inputs(w["Hq"], w["Hkv"], w["N"], w["d"], 0, h, seed=0, **w["gen"])
+                 for h in heads]
+        # head i of the stack is query head heads[i] with its own KV head
+        _ORACLE_INPUTS.clear()
+        _ORACLE_INPUTS[key] = tuple(torch.cat([t[j] for t in drawn], dim=1) for j in range(3))
+    Q, K, V = _ORACLE_INPUTS[key]
+    n_rb = -(-w["N"] // w["Br"])
     cores = cpu_cores()
-
-    def flops_of(units):
-        f = 0.0
-        for _, _, rb in units:
-            rows = min(w["N"], (rb + 1) * w["Br"]) - rb * w["Br"]
-            keys = min(w["N"], (rb + 1) * w["Br"]) if w["causal"] else w["N"]
-            f += 4.0 * rows * keys * w["d"] * (0.5 if w["causal"] else 1.0)
-        return f
 
     def run(units):
         t = time.perf_counter()
-        oracle.prefill(Q, K, V, w["causal"], math.inf, w["Br"], w["Bc"], units=units,
-                       want_exact=False, nthreads=cores)
+        oracle.prefill(Q, K, V, True, math.inf, w["Br"], w["Bc"], units=units, want_exact=False,
+                       nthreads=cores)
         return time.perf_counter() - t
 
-    # calibrate: grow the sample until it takes a quarter of the target time
-    n = min(len(all_units), max(cores, 8))
-    run(all_units[:n])  # first call pays for thread start-up
-    while True:
-        pick = [all_units[i] for i in rng.choice(len(all_units), n, replace=False)]
-        t = run(pick)
-        if t >= target_s / 4 or n >= len(all_units):
-            break
-        n = min(len(all_units), n * 4)
-    n2 = int(min(len(all_units), max(n, n * target_s / max(t, 1e-3))))
-    if n2 > n:
-        pick = [all_units[i] for i in rng.choice(len(all_units), n2, replace=False)]
-        t = run(pick)
-    return flops_of(pick) / t / 1e12, t, len(pick), cores
+    def pick(n):
+        flat = rng.choice(len(heads) * n_rb, n, replace=False)
+        return [(0, int(x) // n_rb, int(x) % n_rb) for x in flat]
+
+    if n_units is None:
+        run(pick(1))  # the first call pays for thread start-up
+        n = 2 * cores
+        t = run(pick(n))
+        n_units = int(min(len(heads) * n_rb, max(cores, n * target_s / max(t, 1e-3))))
+    units = pick(n_units)
+    t = run(units)
+    # dense-equivalent: half of 4 * rows * keys * d per row block under the causal mask
+    f = sum(4.0 * w["Br"] * min(w["N"], (rb + 1) * w["Br"]) * w["d"] * 0.5 for _, _, rb in units)
+    return f / t / 1e12, t, n_units, cores, heads
 
 
 def reference_arm(args, world, rank):
@@ -207,26 +244,27 @@ def reference_arm(args, world, rank):
         return 0
     from block_skipping_softmax_b200 import inputs
 
-    w = inputs.WORKLOADS[MAIN]
-    Q, K, V = inputs.prefill_inputs(w["B"], w["Hq"], w["Hkv"], w["N"], w["d"], seed=0, **w["gen"])
-    # each step: a fresh sample of row blocks sized to ~1.5 s of CPU time
+    w = inputs.WORKLOADS[HEADLINE]
+    # each step: a fresh random sample of row blocks, ~1.5 s of CPU time
     rates, secs = [], []
+    heads = n_units = None
+    cores = 0
     for i in range(args.warmup + args.steps):
-        r, t, n, cores = oracle_sample_rate(w, 1.5, Q, K, V, seed=100 + i)
+        r, t, n_units, cores, heads = oracle_sample_headline(2.0, seed=100 + i, heads=heads,
+                                                             n_units=n_units)
         if i >= args.warmup:
             rates.append(r)
             secs.append(t)
     value = statistics.mean(rates)
+    sample = (f"{n_units} random row blocks (128 queries each, causal) of query heads {heads} of "
+              f"{HEADLINE} per step, {statistics.mean(secs):.1f} s of fp64 CPU work each")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * statistics.mean(secs),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic",
-        "config": {"workload": MAIN, "B": w["B"], "Hq": w["Hq"], "Hkv": w["Hkv"], "N": w["N"],
-                   "d": w["d"], "causal": w["causal"], "Br": w["Br"], "Bc": w["Bc"], "tau": "inf"},
+        "data": "synthetic", "config": headline_config(w, world),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                         "sample": f"{n} random row blocks of {w['Br']} queries per step (of "
-                                   f"{w['B'] * w['Hq'] * (-(-w['N'] // w['Br']))})"},
+                         "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -237,10 +275,10 @@ def reference_arm(args, world, rank):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="own", choices=["own", "reference"])
-    ap.add_argument("--quick", action="store_true", help="skip the extra workloads and the CPU baseline")
+    ap.add_argument("--quick", action="store_true", help="headline, e2e and the five workloads only")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_setup()
@@ -271,6 +309,7 @@ def main():
     peaks, peak_src = load_peaks()
     dev = torch.device("cuda", local)
     stream = torch.cuda.current_stream()
+    steps_x = max(3, args.steps // 4)  # steps of the secondary lines
 
     def barrier():
         if dist:
@@ -329,69 +368,116 @@ def main():
     if rank == 0:
         clocks.start()
 
-    # ---------------- headline: prefill, encoder workload, tau = inf
-    w = inputs.WORKLOADS[MAIN]
-    Qm, Km, Vm = inputs.prefill_inputs(w["B"], w["Hq"], w["Hkv"], w["N"], w["d"], seed=rank, **w["gen"])
-    Q, K, V = Qm.to(dev), Km.to(dev), Vm.to(dev)
-    O = torch.empty_like(Q)
+    configs = {name: {"config": i + 1, "workload": name, "runs": []} for i, name in enumerate(CONFIG_ORDER)}
 
-    def step():
-        bss.prefill(Q, K, V, w["causal"], math.inf, w["Br"], w["Bc"], out=O)
-
-    ms, t0, t1 = timed(step, args.steps, args.warmup, "prefill " + MAIN)
-    flops = dense_flops(w)
-    value = world * flops / (ms * 1e-3) / 1e12
-    achieved = flops / (ms * 1e-3) / 1e12
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": achieved / peaks["bf16_tflops"],
-                "traffic": measured_traffic("prefill_pp_kernel", "prefill_pp_sm100.cu"),
-                "algorithmic_bytes": compulsory_prefill_bytes(w),
-                "peak_source": f"{peak_src} bf16 burst (kernel timed alone)",
-                "kernel": "prefill_pp_kernel<128,64,false> (two 128-row blocks per CTA, persistent)",
-                "algorithmic": "4*B*Hq*N^2*d dense-equivalent FLOPs per launch"}
-    clk = clocks.summary(t0, t1) if rank == 0 else None
-
-    # ---------------- end to end through the public API from pinned host memory
-    Qp, Kp, Vp = Qm.pin_memory(), Km.pin_memory(), Vm.pin_memory()
-    Op = torch.empty_like(Qm).pin_memory()
-
-    def e2e_step():
-        # one public call: host inputs in, host output back; the library cuts
-        # the batch into chunks whose copies overlap the kernels
-        bss.prefill_host(Qp, Kp, Vp, w["causal"], math.inf, w["Br"], w["Bc"], out=Op, stream=stream)
-
-    e2e_steps = max(3, min(args.steps, 20))
-    ms_e2e, _, _ = timed(e2e_step, e2e_steps, 2, "e2e")
-    e2e = {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
-           "h2d_bytes_per_step": Qp.numel() * 2 + Kp.numel() * 2 + Vp.numel() * 2,
-           "d2h_bytes_per_step": Op.numel() * 2, "ms_per_step": ms_e2e,
-           "path": "attn_prefill_host: pinned host -> chunked copies overlapping attn_prefill_ex "
-                   "-> pinned host"}
-    del Qp, Kp, Vp, Op
-
-    # tau = 4 on the same workload, plus its skipped fraction
-    extras = {}
-
-    def prefill_extra(name, wl, Qd, Kd, Vd, tau, steps, warmup):
+    def prefill_run(name, wl, Qd, Kd, Vd, tau, steps, warmup, label=None, record=True):
+        """Time one prefill line; returns its entry (dense and executed
+        TFLOP/s, skipped fraction, latency, fractions of the bf16 peaks)."""
         Od = torch.empty_like(Qd)
-        ms_x, _, _ = timed(lambda: bss.prefill(Qd, Kd, Vd, wl["causal"], tau, wl["Br"], wl["Bc"], out=Od),
-                           steps, warmup, f"{name}@tau={tau}")
+        ms_x, t0, t1 = timed(lambda: bss.prefill(Qd, Kd, Vd, wl["causal"], tau, wl["Br"], wl["Bc"], out=Od),
+                             steps, warmup, label or f"{name}@tau={tau}")
         _, mask = bss.prefill(Qd, Kd, Vd, wl["causal"], tau, wl["Br"], wl["Bc"], out=Od, skip_mask=True)
         mk = mask[mask != 2]
         f = dense_flops(wl)
         skipped = float((mk == 1).float().mean().item())
         visited = mk.numel()
-        # executed MMA FLOPs: every visited tile's QK^T, every kept tile's PV
+        del mask, mk, Od
+        # executed MMA FLOPs: every visited tile's Q K^T, every kept tile's P V
         executed = visited * 2.0 * wl["Br"] * wl["Bc"] * wl["d"] * (2.0 - skipped)
-        extras[f"{name}@tau={tau}"] = {
-            "ms": ms_x, "dense_tflops": f / (ms_x * 1e-3) / 1e12,
-            "executed_tflops": executed / (ms_x * 1e-3) / 1e12,
-            "frac_of_peak": f / (ms_x * 1e-3) / 1e12 / peaks["bf16_tflops"],
-            # a launch of 50 ms or more runs under the power cap: compare it
-            # with the sustained GEMM figure as well
-            "frac_of_sustained_peak": (f / (ms_x * 1e-3) / 1e12 / peaks["bf16_tflops_sustained"]
-                                       if ms_x >= 50.0 else None),
-            "skipped_fraction": skipped, "tiles_visited": visited}
+        tfl = f / (ms_x * 1e-3) / 1e12
+        entry = {"tau": "inf" if math.isinf(tau) else tau, "ms": ms_x, "latency_us": ms_x * 1e3,
+                 "steps": steps, "dense_tflops": tfl,
+                 "executed_tflops": executed / (ms_x * 1e-3) / 1e12,
+                 "frac_of_peak": tfl / peaks["bf16_tflops"],
+                 # a launch of 50 ms or more runs under the power cap: compare it
+                 # with the sustained GEMM figure as well
+                 "frac_of_sustained_peak": tfl / peaks["bf16_tflops_sustained"] if ms_x >= 50.0 else None,
+                 "skipped_fraction": skipped, "tiles_visited": visited,
+                 "gpu_launches": steps}
+        if record:
+            configs[name]["runs"].append(entry)
+        return entry, t0, t1
+
+    # ================= headline: the 70B layer at 128K, tau = inf
+    wh = inputs.WORKLOADS[HEADLINE]
+    # drawn by the GPU's generator (the same recipe; a CPU draw of the 2.1 GB
+    # Q would take minutes)
+    Qh, Kh, Vh = inputs.prefill_inputs(wh["B"], wh["Hq"], wh["Hkv"], wh["N"], wh["d"], seed=rank,
+                                       device=str(dev), **wh["gen"])
+    Oh = torch.empty_like(Qh)
+
+    def step():
+        bss.prefill(Qh, Kh, Vh, wh["causal"], math.inf, wh["Br"], wh["Bc"], out=Oh)
+
+    ms, t0, t1 = timed(step, args.steps, args.warmup, "prefill " + HEADLINE)
+    clk = clocks.summary(t0, t1) if rank == 0 else None
+    flops = dense_flops(wh)
+    achieved = flops / (ms * 1e-3) / 1e12
+    value = world * achieved
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": achieved / peaks["bf16_tflops"],
+                "frac_of_sustained_peak": achieved / peaks["bf16_tflops_sustained"],
+                "sustained_peak": peaks["bf16_tflops_sustained"],
+                "traffic": measured_traffic("prefill_pp_kernel@" + HEADLINE, "prefill_pp_sm100.cu"),
+                "algorithmic_bytes": compulsory_prefill_bytes(wh),
+                "peak_source": f"{peak_src} bf16 burst; the sustained figure (seconds-long GEMM loop "
+                               f"under the power cap) is given beside it",
+                "kernel": "prefill_pp_kernel<128,128,causal> (two 128-row blocks per CTA, persistent)",
+                "algorithmic": "2*B*Hq*N^2*d dense-equivalent FLOPs per launch (causal half of 4*N^2*d "
+                               "per head); one launch per step"}
+    configs[HEADLINE]["runs"].append(
+        {"tau": "inf", "ms": ms, "latency_us": ms * 1e3, "steps": args.steps, "dense_tflops": achieved,
+         "executed_tflops": None, "frac_of_peak": achieved / peaks["bf16_tflops"],
+         "frac_of_sustained_peak": achieved / peaks["bf16_tflops_sustained"], "gpu_launches": args.steps,
+         "skipped_fraction": 0.0, "note": "headline region; tau = inf skips nothing by definition"})
+
+    # ---------------- end to end through the public API, from pinned host memory
+    Qp = torch.empty(Qh.shape, dtype=Qh.dtype, pin_memory=True)
+    Kp = torch.empty(Kh.shape, dtype=Kh.dtype, pin_memory=True)
+    Vp = torch.empty(Vh.shape, dtype=Vh.dtype, pin_memory=True)
+    Op = torch.empty(Qh.shape, dtype=Qh.dtype, pin_memory=True)
+    Qp.copy_(Qh)
+    Kp.copy_(Kh)
+    Vp.copy_(Vh)
+
+    def e2e_step():
+        # one public call: host inputs in, host output back; the library cuts
+        # the layer into chunks of KV-head groups whose copies overlap the kernels
+        bss.prefill_host(Qp, Kp, Vp, wh["causal"], math.inf, wh["Br"], wh["Bc"], out=Op, stream=stream)
+
+    ms_e2e, _, _ = timed(e2e_step, steps_x, 2, "e2e " + HEADLINE)
+    torch.cuda.synchronize()
+    e2e_equal = bool(torch.equal(Op[0, :2].to(dev), Oh[0, :2]))  # the path computes the same output
+    e2e = {"value": world * flops / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOP/s",
+           "h2d_bytes_per_step": Qp.numel() * 2 + Kp.numel() * 2 + Vp.numel() * 2,
+           "d2h_bytes_per_step": Op.numel() * 2, "ms_per_step": ms_e2e, "steps": steps_x,
+           "output_equals_device_path": e2e_equal,
+           "path": "attn_prefill_host: pinned host -> chunks of KV-head groups, copies overlapping "
+                   "attn_prefill_ex -> pinned host"}
+    del Qp, Kp, Vp, Op
+    # tau = 4 on the headline layer, plus its skipped fraction
+    prefill_run(HEADLINE, wh, Qh, Kh, Vh, 4.0, steps_x, 2)
+    del Qh, Kh, Vh, Oh
+    torch.cuda.empty_cache()
+
+    # ================= the other workloads, each at its thresholds
+    ws = inputs.WORKLOADS[SMALL]
+    Qs, Ks, Vs = (t.to(dev) for t in inputs.prefill_inputs(ws["B"], ws["Hq"], ws["Hkv"], ws["N"], ws["d"],
+                                                           seed=rank, **ws["gen"]))
+    for tau in ws["taus"]:
+        prefill_run(SMALL, ws, Qs, Ks, Vs, tau, max(args.steps, 200), args.warmup)
+    configs[SMALL]["note"] = ("4 CTAs on a 148-SM GPU: launch-bound, inputs resident in L2; "
+                              "reported for completeness")
+    del Qs, Ks, Vs
+
+    we = inputs.WORKLOADS[ENCODER]
+    Qm, Km, Vm = inputs.prefill_inputs(we["B"], we["Hq"], we["Hkv"], we["N"], we["d"], seed=rank, **we["gen"])
+    Qe, Ke, Ve = Qm.to(dev), Km.to(dev), Vm.to(dev)
+    del Qm, Km, Vm
+    for tau in we["taus"]:
+        prefill_run(ENCODER, we, Qe, Ke, Ve, tau, args.steps, args.warmup)
+
+    extras = {}
 
     def qk8_extra(name, wl, Qd, Kd, Vd, tau, steps, warmup, int8=False):
         """The 8-bit Q K^T paths: e4m3 (or int8) Q and K, quantised once,
@@ -417,65 +503,63 @@ def main():
         if tau == math.inf:
             ms_q, _, _ = timed(lambda: (quant(Qd, out=(Q8, qs)), quant(Kd, out=(K8, ks))),
                                steps, warmup, f"{name} quantize {tag}")
-            qbytes = (Qd.numel() + Kd.numel()) * 3  # read bf16, write e4m3
+            qbytes = (Qd.numel() + Kd.numel()) * 3  # read bf16, write 8-bit
             entry["quantize_q_and_k_ms"] = ms_q
             entry["quantize_gbs"] = qbytes / (ms_q * 1e-3) / 1e9
         extras[f"{name} {tag}@tau={tau}"] = entry
         del Q8, K8, Od
 
-    prefill_extra(MAIN, w, Q, K, V, math.inf, max(3, args.steps // 4), 3)
-    prefill_extra(MAIN, w, Q, K, V, 4.0, max(3, args.steps // 4), 2)
     if not args.quick:
         # the same batch packed as variable-length sequences ([tokens, H, d],
         # cu_seqlens), the serving layout
-        Qv = Q.permute(0, 2, 1, 3).reshape(-1, w["Hq"], w["d"]).contiguous()
-        Kv = K.permute(0, 2, 1, 3).reshape(-1, w["Hkv"], w["d"]).contiguous()
-        Vv = V.permute(0, 2, 1, 3).reshape(-1, w["Hkv"], w["d"]).contiguous()
+        Qv = Qe.permute(0, 2, 1, 3).reshape(-1, we["Hq"], we["d"]).contiguous()
+        Kv = Ke.permute(0, 2, 1, 3).reshape(-1, we["Hkv"], we["d"]).contiguous()
+        Vv = Ve.permute(0, 2, 1, 3).reshape(-1, we["Hkv"], we["d"]).contiguous()
         Ov = torch.empty_like(Qv)
-        cu = torch.arange(0, w["B"] * w["N"] + 1, w["N"], dtype=torch.int32, device=dev)
-        ms_v, _, _ = timed(lambda: bss.prefill_varlen(Qv, Kv, Vv, cu, w["N"], w["causal"], math.inf,
-                                                      w["Br"], w["Bc"], out=Ov),
-                           max(3, args.steps // 4), 2, f"{MAIN} varlen@tau=inf")
-        extras[f"{MAIN} varlen@tau=inf"] = {
-            "ms": ms_v, "dense_tflops": dense_flops(w) / (ms_v * 1e-3) / 1e12,
-            "frac_of_peak": dense_flops(w) / (ms_v * 1e-3) / 1e12 / peaks["bf16_tflops"],
-            "layout": f"{w['B']} sequences of {w['N']} tokens packed as [tokens, H, d]"}
+        cu = torch.arange(0, we["B"] * we["N"] + 1, we["N"], dtype=torch.int32, device=dev)
+        ms_v, _, _ = timed(lambda: bss.prefill_varlen(Qv, Kv, Vv, cu, we["N"], we["causal"], math.inf,
+                                                      we["Br"], we["Bc"], out=Ov),
+                           steps_x, 2, f"{ENCODER} varlen@tau=inf")
+        extras[f"{ENCODER} varlen@tau=inf"] = {
+            "ms": ms_v, "dense_tflops": dense_flops(we) / (ms_v * 1e-3) / 1e12,
+            "frac_of_peak": dense_flops(we) / (ms_v * 1e-3) / 1e12 / peaks["bf16_tflops"],
+            "layout": f"{we['B']} sequences of {we['N']} tokens packed as [tokens, H, d]"}
         del Qv, Kv, Vv, Ov, cu
-    if not args.quick:
-        qk8_extra(MAIN, w, Q, K, V, math.inf, max(3, args.steps // 4), 2)
-        qk8_extra(MAIN, w, Q, K, V, math.inf, max(3, args.steps // 4), 2, int8=True)
-    del Q, K, V, O
+        qk8_extra(ENCODER, we, Qe, Ke, Ve, math.inf, steps_x, 2)
+        qk8_extra(ENCODER, we, Qe, Ke, Ve, math.inf, steps_x, 2, int8=True)
+    del Qe, Ke, Ve
     torch.cuda.empty_cache()
 
     # ---------------- decode: KV-read GB/s
     wd = inputs.WORKLOADS[DECODE]
-    qh, Kh, Vh = inputs.decode_inputs(wd["B"], wd["Hq"], wd["Hkv"], wd["L"], wd["d"], seed=rank, **wd["gen"])
-    q, Kd, Vd = qh.to(dev), Kh.to(dev), Vh.to(dev)
-    del Kh, Vh
+    qh, Kdh, Vdh = inputs.decode_inputs(wd["B"], wd["Hq"], wd["Hkv"], wd["L"], wd["d"], seed=rank, **wd["gen"])
+    q, Kd, Vd = qh.to(dev), Kdh.to(dev), Vdh.to(dev)
+    del Kdh, Vdh
     o = torch.empty_like(q)
-    decode = {}
     kv_bytes = wd["B"] * wd["Hkv"] * wd["L"] * wd["d"] * 2
+    dec_traffic = measured_traffic("decode_partial_kernel@" + DECODE, "decode_sm100.cu")
     for tau in wd["taus"]:
-        ms_d, d0, d1 = timed(lambda: bss.decode(q, Kd, Vd, tau, out=o), args.steps, args.warmup,
-                             f"decode@tau={tau}")
+        ms_d, _, _ = timed(lambda: bss.decode(q, Kd, Vd, tau, out=o), args.steps, args.warmup,
+                           f"decode@tau={tau}")
         _, mask = bss.decode(q, Kd, Vd, tau, out=o, skip_mask=True)
         kept = 1.0 - float((mask == 1).float().mean().item())
         read = kv_bytes * (1.0 + kept)
         gbs = read / (ms_d * 1e-3) / 1e9
-        decode[f"tau={tau}"] = {
-            "value": world * gbs, "unit": "GB/s", "ms_per_step": ms_d, "latency_us": ms_d * 1000,
-            "dense_equiv_gbs": world * 2 * kv_bytes / (ms_d * 1e-3) / 1e9,
-            "skipped_fraction": 1.0 - kept, "gpu_launches": 2 * args.steps,
+        configs[DECODE]["runs"].append({
+            "tau": "inf" if math.isinf(tau) else tau, "ms": ms_d, "latency_us": ms_d * 1000,
+            "steps": args.steps, "kv_read_gbs": gbs,
+            "dense_equiv_gbs": 2 * kv_bytes / (ms_d * 1e-3) / 1e9, "skipped_fraction": 1.0 - kept,
+            "frac_of_hbm": gbs / peaks["hbm_gbs"], "gpu_launches": 2 * args.steps,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / peaks["hbm_gbs"],
-                         "traffic": measured_traffic("decode_partial_kernel", "decode_sm100.cu"),
+                         "traffic": dec_traffic if math.isinf(tau) else None,
                          "peak_source": f"{peak_src} HBM copy bandwidth",
                          "kernel": "decode_partial_kernel<128,4> + decode_combine_kernel<128>",
                          "algorithmic": "K bytes + kept fraction x V bytes per launch"},
-            "split_len": bss.attn_decode_split_len(wd["B"], wd["Hkv"], wd["L"])}
-    # the decode rule variants (per-head test, sink-seeded splits) at the
-    # thresholds where the skip rule acts
+            "split_len": bss.attn_decode_split_len(wd["B"], wd["Hkv"], wd["L"])})
     if not args.quick:
+        # the decode rule variants (per-head test, sink-seeded splits) at the
+        # thresholds where the skip rule acts
         g = wd["Hq"] // wd["Hkv"]
         ls = bss.attn_decode_split_len(wd["B"], wd["Hkv"], wd["L"])
         n_splits = -(-wd["L"] // ls)
@@ -484,7 +568,7 @@ def main():
                             (bss.RULE_PER_HEAD | bss.RULE_SINK_SEED, "per_head+sink_seed")):
             for tau in (2.0, 4.0):
                 ms_v, _, _ = timed(lambda: bss.decode(q, Kd, Vd, tau, out=o, rule=rule),
-                                   max(3, args.steps // 4), 2, f"decode {rname}@tau={tau}")
+                                   steps_x, 2, f"decode {rname}@tau={tau}")
                 _, mask = bss.decode(q, Kd, Vd, tau, out=o, skip_mask=True, rule=rule)
                 if rule & bss.RULE_PER_HEAD:
                     m4 = mask.view(wd["B"], wd["Hkv"], g, -1)
@@ -498,10 +582,10 @@ def main():
                 read = kv_bytes * (1.0 + v_kept) + seed_bytes
                 gbs = read / (ms_v * 1e-3) / 1e9
                 variants[f"{rname}@tau={tau}"] = {
-                    "value": world * gbs, "unit": "GB/s", "latency_us": ms_v * 1000,
+                    "kv_read_gbs": gbs, "latency_us": ms_v * 1000,
                     "v_tiles_skipped": 1.0 - v_kept, "row_tiles_skipped": row_skip,
-                    "frac_of_hbm": gbs / peaks["hbm_gbs"]}
-        decode["rule_variants"] = variants
+                    "bytes_read": read, "frac_of_hbm": gbs / peaks["hbm_gbs"]}
+        extras["decode_rule_variants"] = variants
         # the same cache as a pool of 64-key pages in shuffled order, read
         # through a block table (the serving layout)
         B_, Hkv_, L_, d_ = wd["B"], wd["Hkv"], wd["L"], wd["d"]
@@ -515,63 +599,76 @@ def main():
         table = perm.view(B_, npg).to(torch.int32).contiguous()
         lens = torch.full((B_,), L_, dtype=torch.int32, device=dev)
         ms_p, _, _ = timed(lambda: bss.decode_paged(q, Kp, Vp, table, lens, L_, math.inf, out=o),
-                           max(3, args.steps // 4), 2, "decode paged@tau=inf")
+                           steps_x, 2, "decode paged@tau=inf")
         gbs = 2 * kv_bytes / (ms_p * 1e-3) / 1e9
-        decode["paged@tau=inf"] = {"value": world * gbs, "unit": "GB/s", "latency_us": ms_p * 1000,
-                                   "frac_of_hbm": gbs / peaks["hbm_gbs"],
-                                   "layout": "pool [B*L/64, Hkv, 64, d], pages in a seeded random order"}
+        extras["decode paged@tau=inf"] = {"kv_read_gbs": gbs, "latency_us": ms_p * 1000,
+                                          "frac_of_hbm": gbs / peaks["hbm_gbs"],
+                                          "layout": "pool [B*L/64, Hkv, 64, d], pages in a seeded random order"}
         del Kp, Vp, table, lens, perm
     del q, Kd, Vd, o
     torch.cuda.empty_cache()
 
-    # ---------------- the causal LLM-layer workloads (timing inputs drawn on the GPU)
+    # ---------------- the causal 8B layer (inputs drawn on the GPU)
+    w8 = inputs.WORKLOADS[LAYER_8B]
+    Q8d, K8d, V8d = inputs.prefill_inputs(w8["B"], w8["Hq"], w8["Hkv"], w8["N"], w8["d"], seed=rank,
+                                          device=str(dev), **w8["gen"])
+    for tau in w8["taus"]:
+        prefill_run(LAYER_8B, w8, Q8d, K8d, V8d, tau, args.steps, args.warmup)
     if not args.quick:
-        for name, steps in (("llama3_8b_causal_N8192", max(3, args.steps // 4)),
-                            ("llama33_70b_causal_N131072", 3)):
-            wl = inputs.WORKLOADS[name]
-            Qd, Kd2, Vd2 = inputs.prefill_inputs(wl["B"], wl["Hq"], wl["Hkv"], wl["N"], wl["d"], seed=rank,
-                                                 device=str(dev), **wl["gen"])
-            for tau in wl["taus"]:
-                prefill_extra(name, wl, Qd, Kd2, Vd2, tau, steps, 1)
-            if name == "llama3_8b_causal_N8192":
-                for tau in (math.inf, 4.0):
-                    qk8_extra(name, wl, Qd, Kd2, Vd2, tau, steps, 1)
-                qk8_extra(name, wl, Qd, Kd2, Vd2, math.inf, steps, 1, int8=True)
-            del Qd, Kd2, Vd2
-            torch.cuda.empty_cache()
+        for tau in (math.inf, 4.0):
+            qk8_extra(LAYER_8B, w8, Q8d, K8d, V8d, tau, steps_x, 2)
+        qk8_extra(LAYER_8B, w8, Q8d, K8d, V8d, math.inf, steps_x, 2, int8=True)
+    del Q8d, K8d, V8d
+    torch.cuda.empty_cache()
+
+    if not args.quick:
+        # Not one of the five workloads: the parity suite's skip-exercising
+        # input (strong sinks: q = 2z + 8u, sink keys 6 sqrt(d) u) at the 8B
+        # layer's shape, where the every-row rule does skip tiles.  The same
+        # input at tau = inf is the time a skip is measured against.
+        gen_s = dict(q_sigma=2.0, q_u=8.0, sink_scale=6.0)
+        Qx, Kx, Vx = inputs.prefill_inputs(w8["B"], w8["Hq"], w8["Hkv"], w8["N"], w8["d"], seed=rank,
+                                           device=str(dev), **gen_s)
+        runs = {}
+        for tau in (math.inf, 4.0, 2.0):
+            e, _, _ = prefill_run(LAYER_8B, w8, Qx, Kx, Vx, tau, args.steps, args.warmup,
+                                  label=f"skip-exercising 8B shape@tau={tau}", record=False)
+            runs["inf" if math.isinf(tau) else str(tau)] = e
+        base = runs["inf"]["ms"]
+        for k, e in runs.items():
+            e["time_vs_tau_inf"] = e["ms"] / base
+            # if a skipped tile cost nothing, time would fall with the P*V half of the work
+            e["pv_work_fraction_left"] = 1.0 - 0.5 * e["skipped_fraction"]
+        extras["skip_exercising_8b_shape"] = {
+            "not_a_baseline_config": True,
+            "input": "B=1, Hq=32, Hkv=8, N=8192, d=128, causal, Br=Bc=128; q = 2z + 8u, "
+                     "sink keys 6 sqrt(d) u (the parity suite's skip-exercising recipe)",
+            "runs": runs}
+        del Qx, Kx, Vx
+        torch.cuda.empty_cache()
     if rank == 0:
         clocks.stop()
 
     cpu_base = None
     if rank == 0 and world == 1 and not args.quick:
-        r, t, n, cores = oracle_sample_rate(w, 10.0, Qm, Km, Vm)
+        r, t, n, cores, heads = oracle_sample_headline(12.0)
         cpu_base = {"value": r, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                    "sample": f"{n} random row blocks ({w['Br']} queries x {w['N']} keys each) of "
-                              f"{MAIN}, {t:.1f} s of fp64 CPU work"}
+                    "sample": f"{n} random row blocks (128 queries each, causal) of query heads "
+                              f"{heads} of {HEADLINE}, {t:.1f} s of fp64 CPU work"}
 
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": MAIN, "B": w["B"], "Hq": w["Hq"], "Hkv": w["Hkv"], "N": w["N"],
-                       "d": w["d"], "causal": w["causal"], "Br": w["Br"], "Bc": w["Bc"], "tau": "inf",
-                       "parallelism": f"replicas x{world} (independent sequences)",
-                       "l2": "inputs 1.07 GB per step > 126 MB L2 (no flush needed)"},
-            "roofline": roofline, "frac_of_tensor_peak": achieved / peaks["bf16_tflops"],
-            "e2e": e2e, "gpu_launches": args.steps, "clocks": clk, "cpu_baseline": cpu_base,
-            "decode": {"metric": "decode KV-read GB/s", "workload": DECODE, **decode},
-            "workloads": extras,
+            "config": headline_config(wh, world),
+            "roofline": roofline, "e2e": e2e, "gpu_launches": args.steps, "clocks": clk,
+            "cpu_baseline": cpu_base,
+            "configs": [configs[n] for n in CONFIG_ORDER],
+            "extras": extras,
             # the pages report no kernel-level figure; their numbers are
             # end-to-end model speedups on other hardware (context only)
-            "pages_context": {
-                "source": "Accelerating Long-Context Inference with Skip Softmax in NVIDIA TensorRT-LLM "
-                          "(Key Points; Detailed Analysis)",
-                "decode_end_to_end_speedup": "about 1.4x, Llama 3.3 70B, NVIDIA GB200 system",
-                "prefill_speedup": "about 40% at 128K context, Llama 3.3 70B, NVIDIA GB200 system",
-                "turboattention_profiling_hardware": "NVIDIA A100 (TurboAttention: Efficient Attention "
-                                                     "Approximation for High-Throughput LLM Serving)",
-            },
+            "pages_context": PAGES_CONTEXT,
             "timing_attempts": attempts_log,
         }
         print(json.dumps(line), flush=True)

@@ -1,5 +1,7 @@
-// Prefill from host memory: the batch is cut into chunks of sequences that
-// flow through two device buffer sets on two streams, so the host-to-device
+// Prefill from host memory: the batch is cut into chunks of KV-head groups
+// (one KV head of one sequence with the g = Hq/Hkv query heads that read it;
+// the groups of consecutive heads are consecutive in memory in every tensor)
+// that flow through two device buffer sets on two streams, so the host-to-device
 // copy of one chunk overlaps the kernel and the device-to-host copy of the
 // previous one (PCIe copies run in both directions at once).  For a caller
 // whose inputs live in (pinned) host memory this makes the whole call bound
@@ -69,9 +71,17 @@ int attn_prefill_host(const void* Qh, const void* Kh, const void* Vh, void* Oh, 
     return ATTN_ERR_INVALID_ARG;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_UNSUPPORTED;
-  const int cb = chunk > 0 ? (chunk < B ? chunk : B) : (B + 7) / 8;  // sequences per chunk
-  const size_t q_seq = static_cast<size_t>(Hq) * N * d * 2;          // bytes of one sequence's Q (and O)
-  const size_t kv_seq = static_cast<size_t>(Hkv) * N * d * 2;
+  // A chunk is `cb` KV-head groups.  Attention of one group touches nothing
+  // outside it, so each chunk runs as a batch of cb "sequences" of g query
+  // heads and one KV head, with the same per-row-block arithmetic (and bit
+  // for bit the same output) as the whole batch on the device.
+  const int g = Hq / Hkv;
+  const long long n_groups_ll = static_cast<long long>(B) * Hkv;
+  if (n_groups_ll > 0x7fffffffLL) return ATTN_ERR_UNSUPPORTED;
+  const int n_groups = static_cast<int>(n_groups_ll);
+  const int cb = chunk > 0 ? (chunk < n_groups ? chunk : n_groups) : (n_groups + 7) / 8;
+  const size_t q_seq = static_cast<size_t>(g) * N * d * 2;  // bytes of one group's Q (and O)
+  const size_t kv_seq = static_cast<size_t>(N) * d * 2;     // of its K (and V)
   const size_t q_b = align256(q_seq * cb), kv_b = align256(kv_seq * cb);
   const size_t set_bytes = 2 * q_b + 2 * kv_b;  // Q, O, K, V
   std::lock_guard<std::mutex> lk(g_mu);
@@ -86,8 +96,8 @@ int attn_prefill_host(const void* Qh, const void* Kh, const void* Vh, void* Oh, 
   const char* kh = static_cast<const char*>(Kh);
   const char* vh = static_cast<const char*>(Vh);
   char* oh = static_cast<char*>(Oh);
-  for (int c = 0, b0 = 0; b0 < B; ++c, b0 += cb) {
-    const int nb = (B - b0 < cb) ? B - b0 : cb;
+  for (int c = 0, b0 = 0; b0 < n_groups; ++c, b0 += cb) {
+    const int nb = (n_groups - b0 < cb) ? n_groups - b0 : cb;
     const int set = c % kSets;
     cudaStream_t s = p.stream[set];
     char* base = static_cast<char*>(p.buf) + set * set_bytes;
@@ -97,7 +107,7 @@ int attn_prefill_host(const void* Qh, const void* Kh, const void* Vh, void* Oh, 
         cudaMemcpyAsync(kd, kh + kv_seq * b0, kv_seq * nb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
         cudaMemcpyAsync(vd, vh + kv_seq * b0, kv_seq * nb, cudaMemcpyHostToDevice, s) != cudaSuccess)
       return ATTN_ERR_CUDA;
-    st = attn_prefill_ex(qd, kd, vd, od, nb, Hq, Hkv, N, d, causal, tau, Br, Bc, s, nullptr);
+    st = attn_prefill_ex(qd, kd, vd, od, nb, g, 1, N, d, causal, tau, Br, Bc, s, nullptr);
     if (st != ATTN_OK) return st;
     if (cudaMemcpyAsync(oh + q_seq * b0, od, q_seq * nb, cudaMemcpyDeviceToHost, s) != cudaSuccess)
       return ATTN_ERR_CUDA;

@@ -100,6 +100,27 @@ def prefill_inputs(B: int, Hq: int, Hkv: int, N: int, d: int, *, seed: int = 0,
     return Q, K, V
 
 
+def prefill_head_inputs(Hq: int, Hkv: int, N: int, d: int, b: int, h: int, *, seed: int = 0,
+                        q_sigma: float = 1.0, q_u: float = 0.0, sink_scale: float | None = None,
+                        n_sinks: int = 4):
+    """Query head (b, h) and its KV head, as [1, 1, N, d] bf16 CPU tensors.
+
+    Bit for bit the slices Q[b, h], K[b, h // (Hq/Hkv)], V[b, h // (Hq/Hkv)]
+    of ``prefill_inputs(...)`` with the same seed and knobs, without drawing
+    the other heads (a very long workload can be sampled one head at a time).
+    """
+    kv = h // (Hq // Hkv)
+    u = unit_vector(d, seed)
+    x = _randn(N, d, derive(seed, "q", b, h)) * q_sigma
+    if q_u:
+        x = x + q_u * u
+    k = _randn(N, d, derive(seed, "k", b, kv))
+    if sink_scale is not None and n_sinks > 0:
+        k[: min(n_sinks, N)] = sink_scale * math.sqrt(d) * u
+    v = _randn(N, d, derive(seed, "v", b, kv))
+    return tuple(t.to(torch.bfloat16).view(1, 1, N, d) for t in (x, k, v))
+
+
 def decode_inputs(B: int, Hq: int, Hkv: int, L: int, d: int, *, seed: int = 0,
                   q_sigma: float = 1.0, q_u: float = 0.0, sink_scale: float | None = None,
                   n_sinks: int = 4):

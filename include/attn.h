@@ -165,8 +165,10 @@ ATTN_API int attn_prefill_qki8(const void* Q8, const void* K8, const float* q_sc
 
 /*
  * Prefill with the inputs and the output in host memory: the batch is cut
- * into chunks of `chunk` sequences (0: B/8 rounded up) that flow through two
- * library-owned device buffer sets on two library streams, so the copy of
+ * into chunks of `chunk` KV-head groups (a group is one KV head of one
+ * sequence and the Hq/Hkv query heads that read it, B*Hkv groups in all;
+ * 0: an eighth of them, rounded up) that flow through two library-owned
+ * device buffer sets on two library streams, so the copy of
  * one chunk to the device overlaps the kernel and the copy back of the
  * previous one.  Qh, Kh, Vh, Oh are host pointers with the layouts of
  * attn_prefill; page-locked (pinned) memory is needed for the copies to

@@ -1,5 +1,6 @@
 """Prefill from host memory (attn_prefill_host): the chunked copy pipeline
-gives exactly the device path's output, for whole and partial last chunks."""
+gives exactly the device path's output, for whole and partial last chunks of
+KV-head groups, including a single sequence cut by KV heads."""
 import math
 
 import pytest
@@ -20,10 +21,12 @@ def lib():
 
 
 @pytest.mark.parametrize("B,Hq,Hkv,N,d,causal,Br,Bc,chunk", [
-    (5, 4, 2, 300, 128, True, 128, 128, 2),     # chunks of 2, 2, 1
+    (5, 4, 2, 300, 128, True, 128, 128, 3),     # 10 groups: chunks of 3, 3, 3, 1
     (8, 4, 4, 512, 128, False, 128, 64, 0),     # default chunking
     (3, 2, 1, 200, 64, True, 64, 64, 1),
     (4, 8, 2, 640, 128, True, 128, 128, 8),     # one chunk
+    (1, 16, 4, 1000, 128, True, 128, 128, 0),   # one sequence, one KV head per chunk
+    (1, 8, 8, 700, 128, False, 128, 64, 3),     # one sequence, chunks of 3, 3, 2 heads
 ])
 def test_host_pipeline_matches_device_path(B, Hq, Hkv, N, d, causal, Br, Bc, chunk):
     Q, K, V = inputs.prefill_inputs(B, Hq, Hkv, N, d, seed=B + N, q_sigma=2.0, q_u=1.0, sink_scale=3.0)
