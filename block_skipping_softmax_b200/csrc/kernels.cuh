@@ -1,5 +1,6 @@
 // Internal launch descriptors shared by the C-ABI layer and the kernels.
 #pragma once
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -38,6 +39,13 @@ struct PrefillLaunch {
 
 int launch_prefill(const PrefillLaunch& a);     // one row block per CTA (any Br)
 int launch_prefill_pp(const PrefillLaunch& a);  // two row blocks per CTA, Br = 128
+// one row block per work item, the softmax warpgroups splitting each key
+// tile's columns: d = 128, Br = 128, fixed-length bf16 batches
+int launch_prefill_split(const PrefillLaunch& a);
+
+// Tensor map over [BH, rows, D] bf16 (d fastest): boxes of 64 columns x
+// box_rows rows, 128-byte swizzle; rows past `rows` read as zeros.
+bool tma_map_bhnd(CUtensorMap* m, const void* base, int BH, int rows, int D, int box_rows);
 
 constexpr int kDecodeTile = 64;  // keys per decode tile
 

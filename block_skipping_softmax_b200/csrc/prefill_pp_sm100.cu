@@ -66,6 +66,8 @@ constexpr float kRescale = 8.0f;  // lazy rescale threshold (log2 units)
 #endif
 constexpr uint32_t kPolyPairs = BSS_POLY_PAIRS;
 
+
+
 // QK8: Q and K arrive as e4m3 (one byte per element, 128-byte rows hold 128
 // columns) and S = Q K^T runs as kind::f8f6f4 MMAs; V and P stay bf16.
 template <int D, int BC, bool QK8 = false>
@@ -131,18 +133,6 @@ struct PPMisc {
   int leave[2][2][4];
 };
 
-__device__ __forceinline__ void named_bar(int id, int count) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
-template <int N>
-__device__ __forceinline__ void reg_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
-}
-template <int N>
-__device__ __forceinline__ void reg_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
-}
 
 __device__ __forceinline__ void pp_give_up(PPMisc* m, int* status, int where) {
   reinterpret_cast<volatile int*>(&m->abort)[0] = 1;
@@ -161,7 +151,8 @@ struct Item {
 
 template <int BC, bool CAUSAL, bool VARLEN>
 __device__ __forceinline__ Item make_item(long long idx, int BH, int n_pairs, int n_rb, int N,
-                                          int Hq, const int* cu_seqlens, int total) {
+                                          int Hq, int Hkv, bool group_major, const int* cu_seqlens,
+                                          int total) {
   Item it;
   int pair;
   if (VARLEN) {
@@ -171,6 +162,18 @@ __device__ __forceinline__ Item make_item(long long idx, int BH, int n_pairs, in
     // clamped, so that a malformed cu_seqlens cannot move a row past the tensors
     it.tok0 = min(max(cu_seqlens[b], 0), total);
     it.len = max(0, min(min(N, cu_seqlens[b + 1] - it.tok0), total - it.tok0));
+  } else if (CAUSAL && group_major) {
+    // KV-head groups one after another (longest pairs first inside a group,
+    // heads fastest): the CTAs in flight share one group's K/V, which then
+    // stays in L2 however long the sequence
+    const int g = Hq / Hkv;
+    const long long per_group = static_cast<long long>(g) * n_pairs;
+    const int grp = static_cast<int>(idx / per_group);
+    const int r = static_cast<int>(idx % per_group);
+    pair = n_pairs - 1 - r / g;
+    it.bh = grp * g + r % g;
+    it.len = N;
+    it.tok0 = 0;
   } else if (CAUSAL) {
     pair = n_pairs - 1 - static_cast<int>(idx / BH);
     it.bh = static_cast<int>(idx % BH);
@@ -314,6 +317,13 @@ __global__ void __launch_bounds__(kPPThreads, 1)
   // more than the mean with plain round robin, 1.6 % with the snake).
   // Non-causal items are all equal and keep plain round robin.  Once an index
   // passes n_items every later one does too.
+  // Causal layers whose KV-head groups hold many items per CTA (long
+  // sequences) go group by group, so the K/V read by the CTAs in flight fits
+  // in L2 (the 128K-token 70B layer: 537 MB of K/V in all, 67 MB per group);
+  // with few items per group, rounds of one group would mix long and short
+  // items and unbalance the CTAs, so heads stay fastest there.
+  const bool group_major =
+      CAUSAL && !VARLEN && static_cast<long long>(g) * n_pairs >= 8LL * gridDim.x;
   auto item_idx = [&](long long k) -> long long {
     const long long G = gridDim.x;
     return k * G + ((CAUSAL && (k & 1)) ? G - 1 - blockIdx.x : blockIdx.x);
@@ -363,7 +373,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       bool alive = true;
       // items counts the non-empty work items (their Q slots); k every index
       for (long long k = 0, idx = item_idx(0); alive && idx < n_items; idx = item_idx(++k)) {
-        const Item it = make_item<BC, CAUSAL, VARLEN>(idx, BH, n_pairs, n_rb, N, Hq, cu_seqlens, total);
+        const Item it = make_item<BC, CAUSAL, VARLEN>(idx, BH, n_pairs, n_rb, N, Hq, Hkv, group_major, cu_seqlens, total);
         if (VARLEN && it.T0 == 0) continue;  // a pair past the end of its sequence
         const int bkv = (it.bh / Hq) * Hkv + (it.bh % Hq) / g;
         const int qs = items % C::kQS;
@@ -432,7 +442,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
       pend.init();
       bool alive = true;
       for (long long k = 0, idx = item_idx(0); alive && idx < n_items; idx = item_idx(++k)) {
-        const Item it = make_item<BC, CAUSAL, VARLEN>(idx, BH, n_pairs, n_rb, N, Hq, cu_seqlens, total);
+        const Item it = make_item<BC, CAUSAL, VARLEN>(idx, BH, n_pairs, n_rb, N, Hq, Hkv, group_major, cu_seqlens, total);
         if (VARLEN && it.T0 == 0) continue;  // a pair past the end of its sequence
         const int bkv = (it.bh / Hq) * Hkv + (it.bh % Hq) / g;
         const int T[2] = {it.T0, it.T1};
@@ -563,7 +573,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           ++cmm;
         };
         for (long long k = 0, idx = item_idx(0); alive && idx < n_items; idx = item_idx(++k)) {
-          const Item it = make_item<BC, CAUSAL, VARLEN>(idx, BH, n_pairs, n_rb, N, Hq, cu_seqlens, total);
+          const Item it = make_item<BC, CAUSAL, VARLEN>(idx, BH, n_pairs, n_rb, N, Hq, Hkv, group_major, cu_seqlens, total);
           if (VARLEN && it.T0 == 0) continue;  // a pair past the end of its sequence
           const int T = t == 0 ? it.T0 : it.T1;
           const int qs = items % C::kQS;
@@ -635,7 +645,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         }
       } else
       for (long long k = 0, idx = item_idx(0); alive && idx < n_items; idx = item_idx(++k)) {
-        const Item it = make_item<BC, CAUSAL, VARLEN>(idx, BH, n_pairs, n_rb, N, Hq, cu_seqlens, total);
+        const Item it = make_item<BC, CAUSAL, VARLEN>(idx, BH, n_pairs, n_rb, N, Hq, Hkv, group_major, cu_seqlens, total);
         if (VARLEN && it.T0 == 0) continue;  // a pair past the end of its sequence
         const int T[2] = {it.T0, it.T1};
         const int qs = items % C::kQS;
@@ -752,7 +762,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
     };
     bool ok = true, failed = false;
     for (long long k = 0, idx = item_idx(0); ok && idx < n_items; idx = item_idx(++k)) {
-      const Item it = make_item<BC, CAUSAL, VARLEN>(idx, BH, n_pairs, n_rb, N, Hq, cu_seqlens, total);
+      const Item it = make_item<BC, CAUSAL, VARLEN>(idx, BH, n_pairs, n_rb, N, Hq, Hkv, group_major, cu_seqlens, total);
       if (VARLEN && it.T0 == 0) continue;  // a pair past the end of its sequence: not a work item
       const int T = t == 0 ? it.T0 : it.T1;
       const int qs = items % C::kQS;
@@ -1109,6 +1119,16 @@ bool pp_map_thd(CUtensorMap* m, const void* base, int H, int tokens, int D, int 
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+}  // namespace
+
+// [BH, rows, D] bf16, d fastest: 64-column boxes of box_rows rows, 128-byte
+// swizzle (shared with the column-split prefill kernel).
+bool tma_map_bhnd(CUtensorMap* m, const void* base, int BH, int rows, int D, int box_rows) {
+  return pp_map(m, base, BH, rows, D, box_rows);
+}
+
+namespace {
+
 template <int D, int BC, bool CAUSAL, bool VARLEN, int QKT>
 int pp_launch(const PrefillLaunch& a) {
   constexpr bool QK8 = QKT != 0;
@@ -1190,6 +1210,14 @@ int launch_prefill_pp(const PrefillLaunch& a) {
     }
     return ATTN_ERR_INVALID_ARG;
   }
+#ifndef BSS_PREFILL_SPLIT
+#define BSS_PREFILL_SPLIT 1
+#endif
+  // d = Bc = 128, fixed length: the column-split kernel (three S buffers
+  // beside one O accumulator; measured faster than two row blocks per CTA,
+  // whose one S buffer per row block serialises S, softmax and P*V).  Bc = 64
+  // keeps two row blocks per CTA with two S buffers each, measured faster.
+  if (BSS_PREFILL_SPLIT && a.d == 128 && a.Bc == 128 && !a.cu_seqlens) return launch_prefill_split(a);
   if (a.d == 128) return a.Bc == 64 ? pp_launch_c<128, 64>(a) : pp_launch_c<128, 128>(a);
   if (a.d == 64) return a.Bc == 64 ? pp_launch_c<64, 64>(a) : pp_launch_c<64, 128>(a);
   return ATTN_ERR_INVALID_ARG;

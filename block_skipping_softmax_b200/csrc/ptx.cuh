@@ -81,6 +81,22 @@ __device__ __forceinline__ bool mbar_drain(uint32_t bar, uint32_t parity, uint64
   }
 }
 
+// Named barrier `id` over `count` threads (a multiple of 32).
+__device__ __forceinline__ void named_bar(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Warp-specialised register budgets: every warp of a warpgroup gives up
+// (dec) or takes (inc) registers to the given per-thread count.
+template <int N>
+__device__ __forceinline__ void reg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void reg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---------------------------------------------------------------- TMA
 // 3-D tiled tensor load into shared memory, completion counted in bytes on
 // an mbarrier.  No multicast.
