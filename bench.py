@@ -418,11 +418,12 @@ def main():
                 "frac": achieved / peaks["bf16_tflops"],
                 "frac_of_sustained_peak": achieved / peaks["bf16_tflops_sustained"],
                 "sustained_peak": peaks["bf16_tflops_sustained"],
-                "traffic": measured_traffic("prefill_pp_kernel@" + HEADLINE, "prefill_pp_sm100.cu"),
+                "traffic": measured_traffic("prefill_split_kernel@" + HEADLINE, "prefill_split_sm100.cu"),
                 "algorithmic_bytes": compulsory_prefill_bytes(wh),
                 "peak_source": f"{peak_src} bf16 burst; the sustained figure (seconds-long GEMM loop "
                                f"under the power cap) is given beside it",
-                "kernel": "prefill_pp_kernel<128,128,causal> (two 128-row blocks per CTA, persistent)",
+                "kernel": "prefill_split_kernel<128,causal> (one 128-row block per work item, softmax "
+                          "warpgroups splitting each key tile's columns, persistent)",
                 "algorithmic": "2*B*Hq*N^2*d dense-equivalent FLOPs per launch (causal half of 4*N^2*d "
                                "per head); one launch per step"}
     configs[HEADLINE]["runs"].append(
@@ -618,6 +619,16 @@ def main():
         for tau in (math.inf, 4.0):
             qk8_extra(LAYER_8B, w8, Q8d, K8d, V8d, tau, steps_x, 2)
         qk8_extra(LAYER_8B, w8, Q8d, K8d, V8d, math.inf, steps_x, 2, int8=True)
+        # part of the exponentials on the FMA-pipe polynomial instead of MUFU
+        for pairs in (4, 8):
+            Od = torch.empty_like(Q8d)
+            ms_p, _, _ = timed(lambda: bss.prefill_poly(Q8d, K8d, V8d, True, math.inf, pairs, out=Od),
+                               steps_x, 2, f"{LAYER_8B} poly{pairs}@tau=inf")
+            tfl = dense_flops(w8) / (ms_p * 1e-3) / 1e12
+            extras[f"{LAYER_8B} poly{pairs}/16@tau=inf"] = {
+                "ms": ms_p, "dense_tflops": tfl, "frac_of_peak": tfl / peaks["bf16_tflops"],
+                "exp2_on_fma_pipes": f"{pairs} of every 16 pairs"}
+            del Od
     del Q8d, K8d, V8d
     torch.cuda.empty_cache()
 

@@ -21,7 +21,7 @@ __all__ = [
     "AttnError", "lib", "attn_prefill", "attn_prefill_ex", "attn_prefill_host", "prefill_host",
     "attn_prefill_varlen", "prefill_varlen", "attn_quantize_e4m3", "quantize_e4m3",
     "attn_prefill_qk8", "prefill_qk8", "attn_quantize_i8", "quantize_i8", "attn_prefill_qki8",
-    "prefill_qki8", "attn_decode", "attn_decode_ex",
+    "prefill_qki8", "attn_prefill_poly", "prefill_poly", "attn_decode", "attn_decode_ex",
     "attn_decode_noalloc", "attn_decode_rule", "attn_decode_paged", "decode_paged", "RULE_GROUP", "RULE_PER_HEAD", "RULE_SINK_SEED",
     "attn_decode_split_len", "attn_decode_tile", "attn_decode_workspace_bytes",
     "attn_set_stream", "attn_sync_status", "attn_last_timeout_site", "attn_set_wait_limit_ms",
@@ -56,6 +56,7 @@ def lib() -> ctypes.CDLL:
         "attn_prefill": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, ci]),
         "attn_prefill_ex": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, ci, vp, vp]),
         "attn_prefill_host": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, ci, ci, vp]),
+        "attn_prefill_poly": (ci, [vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, ci, ci, vp, vp]),
         "attn_prefill_varlen": (ci, [vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, ci, cf, ci, ci, vp, vp]),
         "attn_quantize_e4m3": (ci, [vp, vp, vp, ctypes.c_longlong, ctypes.c_longlong, vp]),
         "attn_prefill_qk8": (ci, [vp, vp, vp, vp, vp, vp, ci, ci, ci, ci, ci, ci, cf, ci, ci, vp, vp]),
@@ -97,6 +98,12 @@ def attn_prefill(Q, K, V, O, B, Hq, Hkv, N, d, causal, tau, Br, Bc) -> int:
 def attn_prefill_ex(Q, K, V, O, B, Hq, Hkv, N, d, causal, tau, Br, Bc, stream=None, skip_mask=None) -> int:
     return lib().attn_prefill_ex(Q, K, V, O, B, Hq, Hkv, N, d, int(causal), float(tau), Br, Bc,
                                  stream, skip_mask)
+
+
+def attn_prefill_poly(Q, K, V, O, B, Hq, Hkv, N, d, causal, tau, Br, Bc, poly_pairs, stream=None,
+                      skip_mask=None) -> int:
+    return lib().attn_prefill_poly(Q, K, V, O, B, Hq, Hkv, N, d, int(causal), float(tau), Br, Bc,
+                                   int(poly_pairs), stream, skip_mask)
 
 
 def attn_prefill_host(Qh, Kh, Vh, Oh, B, Hq, Hkv, N, d, causal, tau, Br, Bc, chunk=0, stream=None) -> int:
@@ -236,6 +243,28 @@ def prefill(Q, K, V, causal: bool, tau: float = math.inf, Br: int = 128, Bc: int
                          causal, tau, Br, Bc, _stream_ptr(stream),
                          mask.data_ptr() if mask is not None else None)
     _check(st, "attn_prefill_ex")
+    return (O, mask) if skip_mask else O
+
+
+def prefill_poly(Q, K, V, causal: bool, tau: float = math.inf, poly_pairs: int = 4, out=None,
+                 skip_mask: bool = False, stream=None):
+    """attn_prefill_poly on bf16 CUDA tensors (d = 128, Br = Bc = 128):
+    poly_pairs of every 16 exponential pairs on the FMA-pipe polynomial."""
+    import torch
+
+    B, Hq, N, d = Q.shape
+    Hkv = K.shape[1]
+    for t in (Q, K, V):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise AttnError(1, "prefill_poly (tensors must be contiguous bf16 CUDA tensors)")
+    O = out if out is not None else torch.empty_like(Q)
+    mask = None
+    if skip_mask:
+        mask = torch.empty(B, Hq, -(-N // 128), -(-N // 128), dtype=torch.uint8, device=Q.device)
+    st = attn_prefill_poly(Q.data_ptr(), K.data_ptr(), V.data_ptr(), O.data_ptr(), B, Hq, Hkv, N, d,
+                           causal, tau, 128, 128, poly_pairs, _stream_ptr(stream),
+                           mask.data_ptr() if mask is not None else None)
+    _check(st, "attn_prefill_poly")
     return (O, mask) if skip_mask else O
 
 

@@ -140,6 +140,40 @@ int attn_prefill_ex(const void* Q, const void* K, const void* V, void* O, int B,
   return Br == 128 ? bss::launch_prefill_pp(a) : bss::launch_prefill(a);
 }
 
+int attn_prefill_poly(const void* Q, const void* K, const void* V, void* O, int B, int Hq,
+                      int Hkv, int N, int d, int causal, float tau, int Br, int Bc, int poly_pairs,
+                      void* stream, uint8_t* skip_mask) {
+  if (poly_pairs != 0 && poly_pairs != 4 && poly_pairs != 8) return ATTN_ERR_INVALID_ARG;
+  if (d != 128 || Br != 128 || Bc != 128) return ATTN_ERR_INVALID_ARG;
+  int st = check_prefill(Q, K, V, O, B, Hq, Hkv, N, d, tau, Br, Bc);
+  if (st != ATTN_OK) return st;
+  int dev = 0;
+  int* status = nullptr;
+  if ((st = device_ready(&dev, &status)) != ATTN_OK) return st;
+  bss::PrefillLaunch a{};
+  a.Q = Q;
+  a.K = K;
+  a.V = V;
+  a.O = O;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.N = N;
+  a.d = d;
+  a.causal = causal ? 1 : 0;
+  a.Br = Br;
+  a.Bc = Bc;
+  a.scale_log2 = kLog2e / std::sqrt(static_cast<float>(d));
+  a.tau_is_inf = std::isinf(tau) ? 1 : 0;
+  a.tau_log2 = a.tau_is_inf ? 0.f : tau * kLog2e;
+  a.skip_mask = skip_mask;
+  a.status = status;
+  a.wait_limit_ns = g_wait_limit_ns;
+  a.stream = static_cast<cudaStream_t>(stream);
+  a.poly_pairs = poly_pairs;
+  return bss::launch_prefill_split(a);
+}
+
 int attn_prefill_varlen(const void* Q, const void* K, const void* V, void* O,
                         const int32_t* cu_seqlens, int B, int max_seqlen, int total_tokens, int Hq,
                         int Hkv, int d, int causal, float tau, int Br, int Bc, void* stream,

@@ -35,6 +35,9 @@ struct PrefillLaunch {
   const float* q_scales;
   const float* k_scales;
   int qk_format;  // with q_scales: 1 e4m3, 2 signed int8
+  // exponential pairs (of every 16) computed by the FMA-pipe polynomial
+  // instead of MUFU: 0, 4 or 8 (column-split kernel, d = Bc = 128)
+  int poly_pairs;
 };
 
 int launch_prefill(const PrefillLaunch& a);     // one row block per CTA (any Br)

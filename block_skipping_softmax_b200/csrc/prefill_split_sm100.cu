@@ -97,12 +97,6 @@ constexpr int kSmemBytes = kOffXm + 2 * 2 * kRows * 4;
 static_assert(kOffLeave + 2 * 8 * 4 <= kOffXm, "misc layout");
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
 
-// Which of the 16 column pairs of each 32-column chunk take the polynomial
-// exp2 instead of MUFU (bit c = pair c).
-#ifndef BSS_SPLIT_POLY_PAIRS
-#define BSS_SPLIT_POLY_PAIRS 0x0000u
-#endif
-constexpr uint32_t kPolyPairs = BSS_SPLIT_POLY_PAIRS;
 
 __device__ __forceinline__ void give_up(volatile int* abort_flag, int* status, int where) {
   *abort_flag = 1;
@@ -167,7 +161,10 @@ struct Pending3 {
 
 }  // namespace
 
-template <int BC, bool CAUSAL>
+// POLY: which of the 16 column pairs of each 32-column chunk take the
+// polynomial exp2 on the FMA pipes instead of MUFU (bit c = pair c; 0 = all
+// on MUFU).
+template <int BC, bool CAUSAL, uint32_t POLY>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_split_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
@@ -628,7 +625,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const float2 x = __ffma2_rn(
                   make_float2(__uint_as_float(u[c0 + 2 * c]), __uint_as_float(u[c0 + 2 * c + 1])), sc2,
                   nm2);
-              const uint32_t w = ((kPolyPairs >> c) & 1u) ? exp2_poly_bf16x2(x)
+              const uint32_t w = ((POLY >> c) & 1u) ? exp2_poly_bf16x2(x)
                                                           : pack_bf16x2(ex2(x.x), ex2(x.y));
               rs2[c & 3] = __fadd2_rn(rs2[c & 3], make_float2(__uint_as_float(w << 16),
                                                               __uint_as_float(w & 0xffff0000u)));
@@ -743,9 +740,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 // --------------------------------------------------------------------- host
 namespace {
 
-template <int BC, bool CAUSAL>
+template <int BC, bool CAUSAL, uint32_t POLY>
 int split_launch(const PrefillLaunch& a) {
-  auto kern = prefill_split_kernel<BC, CAUSAL>;
+  auto kern = prefill_split_kernel<BC, CAUSAL, POLY>;
   static uint64_t ready = 0;  // one bit per device: attributes set and checked
   static int sm_count[64];
   int dev = 0;
@@ -781,8 +778,16 @@ int split_launch(const PrefillLaunch& a) {
 
 int launch_prefill_split(const PrefillLaunch& a) {
   if (a.Br != 128 || a.d != 128 || a.cu_seqlens || a.q_scales) return ATTN_ERR_INVALID_ARG;
-  if (a.Bc == 64) return a.causal ? split_launch<64, true>(a) : split_launch<64, false>(a);
-  if (a.Bc == 128) return a.causal ? split_launch<128, true>(a) : split_launch<128, false>(a);
+  if (a.poly_pairs != 0) {  // polynomial exp2 on 4 or 8 of every 16 pairs; Bc = 128
+    if (a.Bc != 128) return ATTN_ERR_INVALID_ARG;
+    if (a.poly_pairs == 4)
+      return a.causal ? split_launch<128, true, 0x1111u>(a) : split_launch<128, false, 0x1111u>(a);
+    if (a.poly_pairs == 8)
+      return a.causal ? split_launch<128, true, 0x5555u>(a) : split_launch<128, false, 0x5555u>(a);
+    return ATTN_ERR_INVALID_ARG;
+  }
+  if (a.Bc == 64) return a.causal ? split_launch<64, true, 0>(a) : split_launch<64, false, 0>(a);
+  if (a.Bc == 128) return a.causal ? split_launch<128, true, 0>(a) : split_launch<128, false, 0>(a);
   return ATTN_ERR_INVALID_ARG;
 }
 

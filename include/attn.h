@@ -164,6 +164,26 @@ ATTN_API int attn_prefill_qki8(const void* Q8, const void* K8, const float* q_sc
                                void* stream, uint8_t* skip_mask);
 
 /*
+ * Prefill with part of the exponentials computed in software on the FMA pipes
+ * instead of the exponential unit (MUFU): the SAS idea of "TurboAttention:
+ * Efficient Attention Approximation for High-Throughput LLM Serving"
+ * (Technical Deep Dive: SAS), written for base 2 and bf16 probabilities.
+ * 2^x is split into an integer part j = rint(x), added to the exponent field
+ * of the bf16 result, and a degree-3 minimax polynomial of the fraction
+ * f = x - j in [-1/2, 1/2]; the bf16 result is within one ulp of 2^x
+ * correctly rounded.  poly_pairs of every 16 pairs of key columns take the
+ * polynomial (0, 4 or 8; 0 computes every exponential on MUFU and equals
+ * attn_prefill_ex bit for bit); the row sum adds the same bf16 values the
+ * P*V product multiplies, whichever unit made them.  Otherwise as
+ * attn_prefill_ex, for d = 128 and Br = Bc = 128 only.
+ *   Errors: as attn_prefill_ex, plus ATTN_ERR_INVALID_ARG for poly_pairs not
+ *   in {0, 4, 8} or another d, Br or Bc.
+ */
+ATTN_API int attn_prefill_poly(const void* Q, const void* K, const void* V, void* O, int B, int Hq,
+                               int Hkv, int N, int d, int causal, float tau, int Br, int Bc,
+                               int poly_pairs, void* stream, uint8_t* skip_mask);
+
+/*
  * Prefill with the inputs and the output in host memory: the batch is cut
  * into chunks of `chunk` KV-head groups (a group is one KV head of one
  * sequence and the Hq/Hkv query heads that read it, B*Hkv groups in all;

@@ -81,6 +81,19 @@ def test_prefill_rejects_bad_arguments(args):
 
 @no_gpu
 @pytest.mark.parametrize("args", [
+    dict(Q=0), dict(d=64), dict(Bc=64), dict(Br=64, Bc=64), dict(pairs=3), dict(pairs=16),
+    dict(tau=float("nan")), dict(Hq=3, Hkv=2), dict(Q=P + 8),
+])
+def test_prefill_poly_rejects_bad_arguments(args):
+    a = dict(Q=P, K=P, V=P, O=P, B=1, Hq=2, Hkv=1, N=256, d=128, causal=1, tau=1.0, Br=128, Bc=128, pairs=4)
+    a.update(args)
+    st = bss.attn_prefill_poly(a["Q"], a["K"], a["V"], a["O"], a["B"], a["Hq"], a["Hkv"], a["N"], a["d"],
+                               a["causal"], a["tau"], a["Br"], a["Bc"], a["pairs"])
+    assert st == 1
+
+
+@no_gpu
+@pytest.mark.parametrize("args", [
     dict(q=0), dict(L=0), dict(Hq=4, Hkv=3), dict(d=32), dict(tau=float("nan")), dict(tau=-0.5),
     dict(K=P + 4),
 ])
