@@ -84,10 +84,10 @@ constexpr int kOffQ = 0;
 constexpr int kOffK = kOffQ + kQS * kTile;
 constexpr int kOffV = kOffK + kKS * kTile;
 constexpr int kOffMisc = kOffV + kVS * kTile;
-// barriers: k_full[KS], v_full[VS], commit ring[CR], p_full[SB], dec[2][DR],
-// q_full[QS], q_empty[QS], mma_done
-constexpr int kBK = 0, kBV = kBK + kKS, kBC = kBV + kVS, kBP = kBC + kCR, kBD = kBP + kSB,
-              kBQF = kBD + 2 * kDR, kBQE = kBQF + kQS, kBM = kBQE + kQS, kNumBars = kBM + 1;
+// barriers: k_full[KS], v_full[VS], commit ring[CR], p_full[SB], q_full[QS],
+// q_empty[QS], mma_done
+constexpr int kBK = 0, kBV = kBK + kKS, kBC = kBV + kVS, kBP = kBC + kCR, kBQF = kBP + kSB,
+              kBQE = kBQF + kQS, kBM = kBQE + kQS, kNumBars = kBM + 1;
 constexpr int kOffTmem = kOffMisc + kNumBars * 8;
 constexpr int kOffAbort = kOffTmem + 4;
 constexpr int kOffVote = kOffAbort + 4;                 // int [kDR][2][4]
@@ -188,7 +188,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto b_v_full = [&](int s) { return bar0 + 8u * (kBV + s); };
   auto b_cm = [&](int i) { return bar0 + 8u * (kBC + (i % kCR)); };
   auto b_p_full = [&](int b) { return bar0 + 8u * (kBP + b); };
-  auto b_dec = [&](int h, int i) { return bar0 + 8u * (kBD + h * kDR + i); };
   auto b_q_full = [&](int s) { return bar0 + 8u * (kBQF + s); };
   auto b_q_empty = [&](int s) { return bar0 + 8u * (kBQE + s); };
   const uint32_t b_mma_done = bar0 + 8u * kBM;
@@ -204,6 +203,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     return ((*vote_at(i, h, 0) & *vote_at(i, h, 1) & *vote_at(i, h, 2) & *vote_at(i, h, 3)) & 1) ? 0 : 1;
   };
   auto wait_cm = [&](int i) { return mbar_wait(b_cm(i), (i / kCR) & 1, abort_flag, wait_limit_ns); };
+  // all four votes of warpgroup h for decision number dnum (ring slot i) are
+  // in; false if the wait gave up (the abort flag, or the time limit)
+  auto votes_in = [&](int h, int i, int dnum) -> bool {
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t n = 0;; ++n) {
+      bool all = true;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) all = all && ((*vote_at(i, h, w) >> 2) == dnum);
+      if (all) return true;
+      if ((n & 15u) == 15u && (*abort_flag || globaltimer_ns() - t0 > wait_limit_ns)) return false;
+      __nanosleep(96);
+    }
+  };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -231,8 +243,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kVS; ++s) mbar_init(b_v_full(s), 1);
     for (int i = 0; i < kCR; ++i) mbar_init(b_cm(i), 1);
     for (int b = 0; b < kSB; ++b) mbar_init(b_p_full(b), 8);  // one arrival per softmax warp
-    for (int h = 0; h < 2; ++h)
-      for (int i = 0; i < kDR; ++i) mbar_init(b_dec(h, i), 4);  // one per warp of warpgroup h
     for (int s = 0; s < kQS; ++s) {
       mbar_init(b_q_full(s), 1);
       mbar_init(b_q_empty(s), 2);  // one per warpgroup's O store
@@ -314,9 +324,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!tau_is_inf) {
             // every decision is consumed in order; the V of S tile j (or of
             // each kept half) is loaded once some part of it is kept
+            // the softmax warps publish their votes without a barrier
+            // arrival (an arrival is a long-latency step on their path from S
+            // to P); this thread polls the vote words of decision dl, with a
+            // bounded wait
             const int di = dl % kDR;
-            if (!mbar_wait(b_dec(0, di), (dl / kDR) & 1, abort_flag, wait_limit_ns) ||
-                (kHalves && !mbar_wait(b_dec(1, di), (dl / kDR) & 1, abort_flag, wait_limit_ns))) {
+            if (!votes_in(0, di, dl) || (kHalves && !votes_in(1, di, dl))) {
               give_up(abort_flag, status, 3);
               alive = false;
               break;
@@ -553,10 +566,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                             (!row_valid || (mpre != NEG_INF && (mt == NEG_INF || mt < mpre - tau_log2)));
           const bool warp_pass = __all_sync(0xffffffffu, pass) != 0;
           const bool warp_ok = __all_sync(0xffffffffu, waited) != 0;
-          if (lane == 0) {
-            *vote_at(di, h, sw) = (dnum << 2) | (warp_ok ? 0 : 2) | (warp_pass ? 1 : 0);
-            if (kHalves || h == 0) mbar_arrive(b_dec(h, di));
-          }
+          // every lane stores the same word (no divergent branch on the
+          // path from S to P)
+          *vote_at(di, h, sw) = (dnum << 2) | (warp_ok ? 0 : 2) | (warp_pass ? 1 : 0);
           if (warp_pass) {
             // a warp whose rows all pass learns the tile's fate from the
             // other three warps of its warpgroup (stop at the first failure)
