@@ -106,9 +106,9 @@ struct PPCfg {
   static constexpr int kOffV = kOffK + kKS * kKBytes;
   static constexpr int kOffO = kOffV + kVS * kVBytes;
   static constexpr int kOffBar = kOffO + (kOSep ? 2 * kOTile : 0);
-  // k_full[KS], v_full[VS], commit ring[2][CR], p_full[2][SB], dec[2][DR],
+  // k_full[KS], v_full[VS], commit ring[2][CR], p_full[2][SB],
   // q_full[QS], q_empty[QS], mma_done[2]
-  static constexpr int kNumBars = kKS + kVS + 2 * kCR + 2 * kSB + 2 * kDR + 2 * kQS + 2;
+  static constexpr int kNumBars = kKS + kVS + 2 * kCR + 2 * kSB + 2 * kQS + 2;
   static constexpr int kOffMisc = kOffBar + kNumBars * 8;
   static constexpr int kSmemBytes = kOffMisc + 256 + 1024;
   static constexpr int kTmemCols = 512;
@@ -274,9 +274,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
   auto b_cm = [&](int t, int i) { return bar0 + 8u * (kBC + t * kCR + (i % kCR)); };
   constexpr int kBP = kBC + 2 * kCR;
   auto b_p_full = [&](int t, int b) { return bar0 + 8u * (kBP + t * SB + b); };
-  constexpr int kBD = kBP + 2 * SB;
-  auto b_dec = [&](int t, int i) { return bar0 + 8u * (kBD + t * kDR + i); };
-  constexpr int kBQ = kBD + 2 * kDR;
+  constexpr int kBQ = kBP + 2 * SB;
   auto b_q_full = [&](int s) { return bar0 + 8u * (kBQ + s); };
   auto b_q_empty = [&](int s) { return bar0 + 8u * (kBQ + C::kQS + s); };
   // mma_done of MMA issuer 0 and 1 (two issuers at tau = inf)
@@ -296,6 +294,18 @@ __global__ void __launch_bounds__(kPPThreads, 1)
   auto decided_keep = [&](int t, int i) -> int {
     const volatile int* v = misc->vote[t][i];
     return ((v[0] & v[1] & v[2] & v[3]) & 1) ? 0 : 1;
+  };
+  // all four votes of row block t for decision number dnum (ring slot i)
+  // are in; false if the wait gave up (the abort flag, or the time limit)
+  auto votes_in = [&](int t, int i, int dnum) -> bool {
+    const volatile int* v = misc->vote[t][i];
+    const uint64_t t0 = globaltimer_ns();
+    for (uint32_t n = 0;; ++n) {
+      if ((v[0] >> 2) == dnum && (v[1] >> 2) == dnum && (v[2] >> 2) == dnum && (v[3] >> 2) == dnum)
+        return true;
+      if ((n & 15u) == 15u && (*abort_flag || globaltimer_ns() - t0 > wait_limit_ns)) return false;
+      __nanosleep(96);
+    }
   };
   // wait for commit number i of row block t (bounded)
   auto wait_cm = [&](int t, int i) {
@@ -335,7 +345,6 @@ __global__ void __launch_bounds__(kPPThreads, 1)
     for (int t = 0; t < 2; ++t) {
       for (int i = 0; i < kCR; ++i) mbar_init(b_cm(t, i), 1);
       for (int b = 0; b < SB; ++b) mbar_init(b_p_full(t, b), 4);
-      for (int i = 0; i < kDR; ++i) mbar_init(b_dec(t, i), 4);  // one arrival per softmax warp
     }
     for (int s = 0; s < C::kQS; ++s) {
       mbar_init(b_q_full(s), 1);
@@ -496,8 +505,12 @@ __global__ void __launch_bounds__(kPPThreads, 1)
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
             if (!alive || j >= T[t]) continue;
+            // the softmax warps publish their votes without a barrier
+            // arrival (an arrival is a long-latency step on their path from
+            // S to P); this thread polls the four vote words of decision
+            // dl[t] of row block t, with a bounded wait
             const int di = dl[t] % kDR;
-            if (!mbar_wait(b_dec(t, di), (dl[t] / kDR) & 1, abort_flag, wait_limit_ns)) {
+            if (!votes_in(t, di, dl[t])) {
               pp_give_up(misc, status, 3);
               alive = false;
               continue;
@@ -839,10 +852,9 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           const bool warp_pass = __all_sync(0xffffffffu, pass) != 0;
           const bool warp_ok = __all_sync(0xffffffffu, waited) != 0;
           volatile int* vv = misc->vote[t][di];
-          if (lane == 0) {
-            vv[sw] = (dnum << 2) | (warp_ok ? 0 : 2) | (warp_pass ? 1 : 0);
-            mbar_arrive(b_dec(t, di));
-          }
+          // every lane stores the same word (no divergent branch on the path
+          // from S to P)
+          vv[sw] = (dnum << 2) | (warp_ok ? 0 : 2) | (warp_pass ? 1 : 0);
           if (warp_pass) {
             int verdict = 0;  // 1 keep, 2 skip, 3 gave up
             if (lane == 0) {
