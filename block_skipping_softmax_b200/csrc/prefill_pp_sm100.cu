@@ -850,7 +850,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           const bool pass = waited &&
                             (!row_valid || (m_exact != NEG_INF && (mt == NEG_INF || mt < m_exact - tau_log2)));
           const bool warp_pass = __all_sync(0xffffffffu, pass) != 0;
-          const bool warp_ok = __all_sync(0xffffffffu, waited) != 0;
+          const bool warp_ok = waited;  // already the same in every lane (a warp vote)
           volatile int* vv = misc->vote[t][di];
           // every lane stores the same word (no divergent branch on the path
           // from S to P)

@@ -565,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const bool pass = waited && visited &&
                             (!row_valid || (mpre != NEG_INF && (mt == NEG_INF || mt < mpre - tau_log2)));
           const bool warp_pass = __all_sync(0xffffffffu, pass) != 0;
-          const bool warp_ok = __all_sync(0xffffffffu, waited) != 0;
+          const bool warp_ok = waited;  // already the same in every lane (a warp vote)
           // every lane stores the same word (no divergent branch on the
           // path from S to P)
           *vote_at(di, h, sw) = (dnum << 2) | (warp_ok ? 0 : 2) | (warp_pass ? 1 : 0);
