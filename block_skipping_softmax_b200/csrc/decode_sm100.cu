@@ -59,6 +59,8 @@ constexpr int kLag = 2;      // a kept tile's P*V runs kLag iterations after its
 constexpr int kVStages = kLag + 1;
 constexpr int kPRing = kLag + 1;
 constexpr float kRefSlack = 8.f;  // log2 units: probabilities stay below 2^8
+constexpr int kPageChunk = 512;   // paged cache: tiles whose pages are staged at a time
+constexpr int kPageSlots = 2 * kPageChunk;
 
 template <int D, int G>
 struct DecCfg {
@@ -90,6 +92,9 @@ struct DecCfg {
   static constexpr int kOffBar = kOffMisc + 16;
   static constexpr int kSmemUsed = kOffBar + 8 * (kKStages + kVStages + 1);  // + sink-seed tile
   static constexpr int kSmemBytes = kSmemUsed + 1024;  // room to align the base
+  // paged cache only: int [kPageSlots] pages of the split's tiles
+  static constexpr int kOffTab = (kSmemUsed + 15) / 16 * 16;
+  static constexpr int kSmemBytesPaged = kOffTab + kPageSlots * 4 + 1024;
   static_assert(G <= kP, "a lane ends the butterfly with one row");
   static_assert(kSIters >= 1 && kKPI * kSIters == kKeysPerWarp, "score lane layout");
   static_assert(kKeyMajor || kKPI == 8, "qd-major lanes need eight keys per instruction");
@@ -207,20 +212,39 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
     }
   }
 
+  // Paged: the pages of the split's tiles are staged in shared memory (tile
+  // k of the split in slot k % kPageSlots) by all threads, kPageChunk at a
+  // time and a whole chunk before any copy needs them, so the thread that
+  // issues the copies never reads the block table itself: a table read on
+  // that path (an L2 round trip per tile under full HBM load) held every
+  // warp at the next barrier.  Entries past the split's last tile are never
+  // read (t_end <= the tiles the table row addresses).
+  int* pg_tab = reinterpret_cast<int*>(smem + C::kOffTab);
+  auto stage_pages = [&](int k0) {  // tiles k0 .. k0 + kPageChunk - 1 (those < nt)
+    const int* bt_row = block_table + static_cast<size_t>(b) * max_pages + t_begin;
+    const int k1 = min(nt, k0 + kPageChunk);
+    for (int k = k0 + tid; k < k1; k += kDecThreads) pg_tab[k % kPageSlots] = bt_row[k];
+  };
+
   // one tile = kPanels TMA boxes of 64 columns x 64 keys; rows past L read as
   // zeros.  Paged: tile t of this sequence is page block_table[b][t], whose
-  // 64 keys of KV head kv are row (page * Hkv + kv) of the page pool.
-  auto issue = [&](uint32_t dst, const CUtensorMap* map, uint32_t bar, int t) {
+  // 64 keys of KV head kv are row (page * Hkv + kv) of the page pool; the
+  // caller passes the page (unused for the contiguous cache).
+  auto issue = [&](uint32_t dst, const CUtensorMap* map, uint32_t bar, int t, int page) {
     mbar_arrive_expect_tx(bar, C::kTileBytes);
     int c1 = t * kDecodeTile, c2 = bh;
     if constexpr (PAGED) {
       c1 = 0;
-      c2 = block_table[static_cast<size_t>(b) * max_pages + t] * Hkv + kv;
+      c2 = page * Hkv + kv;
     }
 #pragma unroll
     for (int p = 0; p < C::kPanels; ++p)
       tma_load_3d(dst + p * C::kPanelBytes, map, bar, p * 64, c1, c2);
   };
+  if constexpr (PAGED) {  // chunks 0 and 1, published by the barrier below
+    stage_pages(0);
+    stage_pages(kPageChunk);
+  }
 
   if (tid == 0) {
     for (int s = 0; s < kKStages; ++s) mbar_init(b_k_full(s), 1);
@@ -234,7 +258,8 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
   int k_issued = 0, v_issued = 0;
   if (tid == 0) {
     for (int i = 0; i < kKStages && i < nt; ++i) {
-      issue(sbase + C::kOffK + i * C::kTileBytes, &tmK, b_k_full(i), t_begin + i);
+      issue(sbase + C::kOffK + i * C::kTileBytes, &tmK, b_k_full(i), t_begin + i,
+            PAGED ? pg_tab[i] : 0);
       ++k_issued;
     }
   }
@@ -345,7 +370,8 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
   bool seed_issued = false;
   if (seeded && t_begin > 0) {
     if (tid == 0) {
-      issue(sbase + C::kOffV, &tmK, b_seed, 0);
+      issue(sbase + C::kOffV, &tmK, b_seed, 0,
+            PAGED ? block_table[static_cast<size_t>(b) * max_pages] : 0);
       seed_issued = true;
     }
     const bool got = mbar_wait(b_seed, 0, never, wait_limit_ns);
@@ -381,6 +407,16 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
     // ---------------- B: decision for tile i, taken identically by every warp
     bool keep_i = false;
     if (i < nt) {
+      // paged: the pages of this iteration's copies (V of tile i, K of tile
+      // i + kKStages) are read here, beside the row maxima, by every thread,
+      // so the issuing thread does not wait for them after the decision
+      // (when the other warps' P*V loads fill the shared-memory pipe, and
+      // every warp waits for the issuing one at the next barrier)
+      int pg_v = 0, pg_k = 0;
+      if constexpr (PAGED) {
+        pg_v = lds_s32_now(sbase + C::kOffTab + 4u * (i % kPageSlots));
+        pg_k = lds_s32_now(sbase + C::kOffTab + 4u * ((i + kKStages) % kPageSlots));
+      }
       const float* wb = wmax + (i & 1) * kWarps * G;
       float mt = lane < n_dec ? wb[lane] : NEG_INF;
       if constexpr (G == 8) mt = fmaxf(mt, wb[lane + 32]);
@@ -431,15 +467,20 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
           // test support: the first copy can be withheld, so that every wait
           // for it runs out and the timeout path is exercised
           if (!(withhold_v && v_issued == 0))
-            issue(sbase + C::kOffV + vs * C::kTileBytes, &tmV, b_v_full(vs), t);
+            issue(sbase + C::kOffV + vs * C::kTileBytes, &tmV, b_v_full(vs), t, pg_v);
           ++v_issued;
         }
         if (i + kKStages < nt) {  // every thread has finished reading K slot i % kKStages
           const int ks = i % kKStages;
-          issue(sbase + C::kOffK + ks * C::kTileBytes, &tmK, b_k_full(ks), t + kKStages);
+          issue(sbase + C::kOffK + ks * C::kTileBytes, &tmK, b_k_full(ks), t + kKStages, pg_k);
           ++k_issued;
         }
       }
+      // chunk c = i / kPageChunk starts: stage chunk c + 1 into the slots of
+      // chunk c - 1, whose last copy (tile i - 1's V) was issued before the
+      // barrier above; chunk c + 1 is first read kPageChunk - kKStages
+      // barriers later
+      if (PAGED && i >= kPageChunk && i % kPageChunk == 0) stage_pages(i + kPageChunk);
     }
     kept_bits = (kept_bits << 1) | (keep_i ? 1u : 0u);
 
@@ -637,11 +678,12 @@ template <int D, int G, int RULE, bool PAGED>
 int launch_dgrp(const DecodeLaunch& a) {
   using C = DecCfg<D, G>;
   auto kern = decode_partial_kernel<D, G, RULE, PAGED>;
+  constexpr int smem_bytes = PAGED ? C::kSmemBytesPaged : C::kSmemBytes;
   static uint64_t attr_done = 0;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
   if (dev < 64 && !(attr_done >> dev & 1)) {
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes) !=
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_bytes) !=
         cudaSuccess)
       return ATTN_ERR_CUDA;
     attr_done |= uint64_t(1) << dev;
@@ -655,7 +697,7 @@ int launch_dgrp(const DecodeLaunch& a) {
     return ATTN_ERR_CUDA;
   }
   dim3 grid(a.n_splits, a.Hkv, a.B);
-  kern<<<grid, kDecThreads, C::kSmemBytes, a.stream>>>(
+  kern<<<grid, kDecThreads, smem_bytes, a.stream>>>(
       mk, mv, static_cast<const __nv_bfloat16*>(a.q), a.o_part, a.lse_part, a.skip_mask,
       a.status, a.Hq, a.Hkv, a.L, a.split_len, a.n_splits, a.scale_log2, a.tau_log2,
       a.tau_is_inf, a.wait_limit_ns, a.withhold_v, a.block_table, a.seq_lens, a.max_pages);

@@ -97,6 +97,14 @@ __device__ __forceinline__ void reg_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
+// A shared-memory load the compiler keeps where it is written (it is not
+// sunk towards its use), so its latency overlaps the code that follows.
+__device__ __forceinline__ int lds_s32_now(uint32_t addr) {
+  int v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(addr));
+  return v;
+}
+
 // ---------------------------------------------------------------- TMA
 // 3-D tiled tensor load into shared memory, completion counted in bytes on
 // an mbarrier.  No multicast.

@@ -111,6 +111,58 @@ def test_paged_identity_table_equals_contiguous_bitwise():
         assert torch.equal(a, p)
 
 
+def test_paged_long_splits_refill_staged_pages():
+    """One split per sequence (37 x 8 KV heads fill the 296 resident CTAs)
+    of 1032 tiles: the kernel stages a split's pages 512 at a time, so this
+    split refills them inside its tile loop.  Full lengths in a shuffled pool
+    agree bit for bit with the contiguous cache; ragged sequences, whose
+    unowned key slots hold NaN, agree with the oracle."""
+    B, Hkv, Hq, d = 37, 8, 8, 64
+    npg = 1032
+    L = npg * PAGE - 17
+    Ls = bss.attn_decode_split_len(B, Hkv, L)
+    assert Ls >= L, "one split per sequence"
+    gen = torch.Generator(device="cuda").manual_seed(3)
+    q = torch.randn(B, Hq, d, generator=gen, device="cuda").to(torch.bfloat16)
+    K = torch.randn(B, Hkv, npg * PAGE, d, generator=gen, device="cuda").to(torch.bfloat16)
+    V = torch.randn(B, Hkv, npg * PAGE, d, generator=gen, device="cuda").to(torch.bfloat16)
+    K[:, :, L:] = 0  # the contiguous cache is L long: rows past L read as zeros there
+    V[:, :, L:] = 0
+    perm = torch.randperm(B * npg, generator=torch.Generator().manual_seed(5)).cuda()
+    Kp = torch.empty(B * npg, Hkv, PAGE, d, dtype=torch.bfloat16, device="cuda")
+    Vp = torch.empty_like(Kp)
+    Kp[perm] = K.view(B, Hkv, npg, PAGE, d).permute(0, 2, 1, 3, 4).reshape(B * npg, Hkv, PAGE, d)
+    Vp[perm] = V.view(B, Hkv, npg, PAGE, d).permute(0, 2, 1, 3, 4).reshape(B * npg, Hkv, PAGE, d)
+    table = perm.view(B, npg).to(torch.int32).contiguous()
+    full = torch.full((B,), L, dtype=torch.int32, device="cuda")
+    a = bss.decode(q, K[:, :, :L].contiguous(), V[:, :, :L].contiguous(), math.inf)
+    p = bss.decode_paged(q, Kp, Vp, table, full, L, math.inf)
+    assert bss.attn_sync_status() == 0
+    assert torch.equal(a, p)
+    # ragged: sequence 1 ends inside the second staged chunk, sequence 2
+    # inside the first; their unowned slots hold NaN and their table rows end
+    # in invalid entries
+    lens = [L, 700 * PAGE + 5, 600] + [L] * (B - 3)
+    for b in (1, 2):
+        n = lens[b]
+        used = -(-n // PAGE)
+        pages = table[b, :used].long()
+        Kp[pages[-1], :, n - (used - 1) * PAGE:] = float("nan")
+        Vp[pages[-1], :, n - (used - 1) * PAGE:] = float("nan")
+        Kp[table[b, used:].long()] = float("nan")
+        Vp[table[b, used:].long()] = float("nan")
+        table[b, used:] = -1
+    sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    o = bss.decode_paged(q, Kp, Vp, table, sl, L, math.inf)
+    assert bss.attn_sync_status() == 0
+    assert torch.equal(o[0], a[0])
+    for b in (1, 2):
+        n = lens[b]
+        r = oracle.decode(q[b:b + 1].cpu(), K[b:b + 1, :, :n].cpu().contiguous(),
+                          V[b:b + 1, :, :n].cpu().contiguous(), math.inf, Ls, PAGE, want_exact=False)
+        compare_outputs(o[b:b + 1].cpu(), r["o"], np.ones(r["o"].shape, bool))
+
+
 def test_paged_argument_errors():
     q = torch.zeros(1, 4, 128, dtype=torch.bfloat16, device="cuda")
     Kp = torch.zeros(2, 1, PAGE, 128, dtype=torch.bfloat16, device="cuda")
