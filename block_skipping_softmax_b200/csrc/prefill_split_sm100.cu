@@ -163,13 +163,15 @@ struct Pending3 {
 
 // POLY: which of the 16 column pairs of each 32-column chunk take the
 // polynomial exp2 on the FMA pipes instead of MUFU (bit c = pair c; 0 = all
-// on MUFU).
-template <int BC, bool CAUSAL, uint32_t POLY>
+// on MUFU).  SKIP: tau is finite, so the kernel takes the skip test; with
+// tau = inf it holds no trace of it (the test's branches alone cost the
+// softmax loop about 6 % in scheduling).
+template <int BC, bool CAUSAL, uint32_t POLY, bool SKIP>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_split_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                          const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                          uint8_t* __restrict__ skip_mask, int* __restrict__ status, int B, int Hq,
-                         int Hkv, int N, float scale_log2, float tau_log2, int tau_is_inf,
+                         int Hkv, int N, float scale_log2, float tau_log2,
                          unsigned long long wait_limit_ns) {
   static_assert(BC == 64 || BC == 128, "skip granularity");
   constexpr bool kHalves = BC == 64;  // two rule tiles per S tile
@@ -321,7 +323,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; alive && j < it.T; ++j) {
           bool keepA = true;
           bool keepB = !kHalves || 2 * j + 1 < it.T64;
-          if (!tau_is_inf) {
+          if (SKIP) {
             // every decision is consumed in order; the V of S tile j (or of
             // each kept half) is loaded once some part of it is kept
             // the softmax warps publish their votes without a barrier
@@ -329,13 +331,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             // to P); this thread polls the vote words of decision dl, with a
             // bounded wait
             const int di = dl % kDR;
-            if (!votes_in(0, di, dl) || (kHalves && !votes_in(1, di, dl))) {
+            if (!votes_in(0, di, dl) || !votes_in(1, di, dl)) {
               give_up(abort_flag, status, 3);
               alive = false;
               break;
             }
             ++dl;
-            keepA = decided_keep(0, di);
+            keepA = kHalves ? decided_keep(0, di) : (decided_keep(0, di) | decided_keep(1, di));
             keepB = kHalves ? (keepB && decided_keep(1, di)) : keepA;
           }
           if (!keepA && !keepB) continue;
@@ -346,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // tiles j - SB and earlier (items are SB apart in the running
             // tile number).  Those commits are not waited for: after a run of
             // skipped tiles their ring slot may have been reused.
-            const bool known_done = !tau_is_inf && pend.g[0] + kSB < gbase + j;
+            const bool known_done = SKIP && pend.g[0] + kSB < gbase + j;
             if (!known_done && !wait_cm(pend.c[0])) {
               give_up(abort_flag, status, 4);
               alive = false;
@@ -442,9 +444,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           // every softmax warp wrote its vote before arriving on p_full
           bool keepA = true;
           bool keepB = !kHalves || 2 * j + 1 < it.T64;
-          if (!tau_is_inf) {
+          if (SKIP) {
             const int di = dc % kDR;
-            keepA = decided_keep(0, di);
+            keepA = kHalves ? decided_keep(0, di) : (decided_keep(0, di) | decided_keep(1, di));
             keepB = kHalves ? (keepB && decided_keep(1, di)) : keepA;
           }
           ++dc;
@@ -547,21 +549,45 @@ __global__ void __launch_bounds__(kThreads, 1)
               m4[q] = fmax3(m4[q], __uint_as_float(u[c + 2 * q]), __uint_as_float(u[c + 2 * q + 1]));
           mh = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * sl2;  // -inf stays -inf
         }
-        const float mo = exchange(mh);
-        const float mA = h == 0 ? mh : mo;
-        const float mB = h == 0 ? mo : mh;
-        // ---- skip test.  BC = 128: the S tile, with its maximum max(mA, mB);
-        // both warpgroups hold the same row values and reach the same
-        // decision.  BC = 64: warpgroup h decides its own half, tile 2j + h,
-        // whose running maximum includes half A when h = 1.
+        // ---- skip test.  BC = 128: the S tile, whose maximum is max(mA,
+        // mB).  max(mA, mB) < x exactly when mA < x and mB < x, so each
+        // warp votes on its own half of its rows before the exchange (the
+        // running maximum m_exact is the same in the two threads of a row),
+        // and the exchange's barrier makes all eight votes visible: every
+        // warp reads the tile's fate without waiting for another.  BC = 64:
+        // warpgroup h decides its own half, tile 2j + h, whose running
+        // maximum includes half A when h = 1 (known after the exchange).
         const int di = dcount % kDR;
         const int dnum = dcount;
         ++dcount;
         const bool visited = !kHalves || 2 * j + h < it.T64;
+        bool warp_pass = false;
+        if constexpr (!kHalves && SKIP) {
+          const bool pass = waited && (!row_valid || (m_exact != NEG_INF &&
+                                                      (mh == NEG_INF || mh < m_exact - tau_log2)));
+          warp_pass = __all_sync(0xffffffffu, pass) != 0;
+          // every lane stores the same word (no divergent branch on the path
+          // from S to P); waited is the same in every lane
+          *vote_at(di, h, sw) = (dnum << 2) | (waited ? 0 : 2) | (warp_pass ? 1 : 0);
+        }
+        const float mo = exchange(mh);
+        const float mA = h == 0 ? mh : mo;
+        const float mB = h == 0 ? mo : mh;
         bool skip = false;
-        if (!tau_is_inf) {
-          const float mt = kHalves ? mh : fmaxf(mA, mB);
-          const float mpre = (kHalves && h == 1) ? fmaxf(m_exact, mA) : m_exact;
+        if constexpr (!kHalves && SKIP) {
+          // a warp with a failing row knows the tile is kept; a warp whose
+          // rows all pass reads the eight votes, all in since the exchange's
+          // barrier: skipped iff every warp's rows pass in both halves (a
+          // warp that gave up votes keep).  Vote words [di][h][w].
+          if (warp_pass) {
+            int all = 1;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) all &= vote[di * 8 + w];
+            skip = (all & 1) != 0;
+          }
+        } else if (kHalves && SKIP) {
+          const float mt = mh;
+          const float mpre = h == 1 ? fmaxf(m_exact, mA) : m_exact;
           const bool pass = waited && visited &&
                             (!row_valid || (mpre != NEG_INF && (mt == NEG_INF || mt < mpre - tau_log2)));
           const bool warp_pass = __all_sync(0xffffffffu, pass) != 0;
@@ -752,9 +778,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 // --------------------------------------------------------------------- host
 namespace {
 
-template <int BC, bool CAUSAL, uint32_t POLY>
-int split_launch(const PrefillLaunch& a) {
-  auto kern = prefill_split_kernel<BC, CAUSAL, POLY>;
+template <int BC, bool CAUSAL, uint32_t POLY, bool SKIP>
+int split_launch_t(const PrefillLaunch& a) {
+  auto kern = prefill_split_kernel<BC, CAUSAL, POLY, SKIP>;
   static uint64_t ready = 0;  // one bit per device: attributes set and checked
   static int sm_count[64];
   int dev = 0;
@@ -781,9 +807,13 @@ int split_launch(const PrefillLaunch& a) {
   const long long n_items = static_cast<long long>(a.B) * a.Hq * ((a.N + kRows - 1) / kRows);
   const int grid = static_cast<int>(n_items < sm_count[dev] ? n_items : sm_count[dev]);
   kern<<<grid, kThreads, kSmemBytes, a.stream>>>(mq, mk, mv, mo, a.skip_mask, a.status, a.B, a.Hq,
-                                                 a.Hkv, a.N, a.scale_log2, a.tau_log2, a.tau_is_inf,
-                                                 a.wait_limit_ns);
+                                                 a.Hkv, a.N, a.scale_log2, a.tau_log2, a.wait_limit_ns);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int BC, bool CAUSAL, uint32_t POLY>
+int split_launch(const PrefillLaunch& a) {
+  return a.tau_is_inf ? split_launch_t<BC, CAUSAL, POLY, false>(a) : split_launch_t<BC, CAUSAL, POLY, true>(a);
 }
 
 }  // namespace
