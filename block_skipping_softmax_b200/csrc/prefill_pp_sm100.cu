@@ -240,14 +240,16 @@ struct Pending3 {
 }  // namespace
 
 // QKT: Q K^T operand format, 0 bf16, 1 e4m3 (f32 scores), 2 signed int8
-// (int32 scores)
-template <int D, int BC, bool CAUSAL, bool VARLEN, int QKT>
+// (int32 scores).  SKIP: tau is finite, so the kernel takes the skip test;
+// with tau = inf it holds no trace of it (the test's branches alone cost the
+// softmax loop several per cent in scheduling).
+template <int D, int BC, bool CAUSAL, bool VARLEN, int QKT, bool SKIP>
 __global__ void __launch_bounds__(kPPThreads, 1)
     prefill_pp_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                       const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmO,
                       __nv_bfloat16* __restrict__ O,
                       uint8_t* __restrict__ skip_mask, int* __restrict__ status, int B, int Hq,
-                      int Hkv, int N, float scale_log2, float tau_log2, int tau_is_inf,
+                      int Hkv, int N, float scale_log2, float tau_log2,
                       unsigned long long wait_limit_ns, const int* __restrict__ cu_seqlens,
                       int total, const float* __restrict__ q_scales,
                       const float* __restrict__ k_scales) {
@@ -287,7 +289,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
   // finite tau the V loads depend on both row blocks' decisions and warp 1
   // issues for both.  With one S buffer per row block (Bc = 128 at d = 128)
   // the single issuer's fixed alternation measured faster, so it stays.
-  const bool dual = tau_is_inf != 0 && SB == 2;
+  constexpr bool dual = !SKIP && SB == 2;
   PPMisc* misc = reinterpret_cast<PPMisc*>(smem + C::kOffMisc);
   volatile int* abort_flag = &misc->abort;
   // keep (1) or skip (0) from the four vote words of one decision
@@ -463,7 +465,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             // earlier (items are SB apart in g).  Those commits are not
             // waited for, since their ring slot may have been reused after a
             // run of skipped tiles.
-            const bool known_done = !tau_is_inf && pend.g[0] + SB < gbase + j;
+            const bool known_done = SKIP && pend.g[0] + SB < gbase + j;
             if (!known_done && ((pend.c0[0] >= 0 && !wait_cm(0, pend.c0[0])) ||
                                 (pend.c1[0] >= 0 && !wait_cm(1, pend.c1[0]))))
               return false;
@@ -492,7 +494,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
           return true;
         };
         for (int j = 0; alive && j < it.Tmax; ++j) {
-          if (tau_is_inf) {
+          if (!SKIP) {
             if (!issue_v(j)) {
               pp_give_up(misc, status, 4);
               alive = false;
@@ -702,7 +704,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
             ++pc[t];
             tc_fence_after();
             // every warp wrote its vote before arriving on p_full
-            const int keep = tau_is_inf ? 1 : decided_keep(t, dc[t] % kDR);
+            const int keep = SKIP ? decided_keep(t, dc[t] % kDR) : 1;
             ++dc[t];
             if (keep) {
               if (!v_used) {
@@ -846,7 +848,7 @@ __global__ void __launch_bounds__(kPPThreads, 1)
         const int dnum = dcount;
         ++dcount;
         bool skip = false;
-        if (!tau_is_inf) {  // with tau = inf every tile is kept and nobody reads votes
+        if constexpr (SKIP) {  // with tau = inf every tile is kept and nobody reads votes
           const bool pass = waited &&
                             (!row_valid || (m_exact != NEG_INF && (mt == NEG_INF || mt < m_exact - tau_log2)));
           const bool warp_pass = __all_sync(0xffffffffu, pass) != 0;
@@ -1141,11 +1143,11 @@ bool tma_map_bhnd(CUtensorMap* m, const void* base, int BH, int rows, int D, int
 
 namespace {
 
-template <int D, int BC, bool CAUSAL, bool VARLEN, int QKT>
-int pp_launch(const PrefillLaunch& a) {
+template <int D, int BC, bool CAUSAL, bool VARLEN, int QKT, bool SKIP>
+int pp_launch_t(const PrefillLaunch& a) {
   constexpr bool QK8 = QKT != 0;
   using C = PPCfg<D, BC, QK8>;
-  auto kern = prefill_pp_kernel<D, BC, CAUSAL, VARLEN, QKT>;
+  auto kern = prefill_pp_kernel<D, BC, CAUSAL, VARLEN, QKT, SKIP>;
   static uint64_t ready = 0;  // one bit per device: attributes set and checked
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return ATTN_ERR_CUDA;
@@ -1192,9 +1194,14 @@ int pp_launch(const PrefillLaunch& a) {
   const int grid = static_cast<int>(n_items < sm_count[dev] ? n_items : sm_count[dev]);
   kern<<<grid, kPPThreads, C::kSmemBytes, a.stream>>>(
       mq, mk, mv, mo, static_cast<__nv_bfloat16*>(a.O), a.skip_mask, a.status, a.B, a.Hq, a.Hkv, a.N,
-      a.scale_log2, a.tau_log2, a.tau_is_inf, a.wait_limit_ns, a.cu_seqlens, a.total, a.q_scales,
-      a.k_scales);
+      a.scale_log2, a.tau_log2, a.wait_limit_ns, a.cu_seqlens, a.total, a.q_scales, a.k_scales);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+template <int D, int BC, bool CAUSAL, bool VARLEN, int QKT>
+int pp_launch(const PrefillLaunch& a) {
+  return a.tau_is_inf ? pp_launch_t<D, BC, CAUSAL, VARLEN, QKT, false>(a)
+                      : pp_launch_t<D, BC, CAUSAL, VARLEN, QKT, true>(a);
 }
 
 template <int D, int BC>
