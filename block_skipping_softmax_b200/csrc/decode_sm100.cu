@@ -137,14 +137,16 @@ __device__ __forceinline__ void load_row_floats(const float* p, float (&v)[G]) {
 
 }  // namespace
 
-template <int D, int G, int RULE, bool PAGED>
+// SKIP: tau is finite, so the kernel takes the skip test; with tau = inf it
+// holds no trace of it.
+template <int D, int G, int RULE, bool PAGED, bool SKIP>
 __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
     decode_partial_kernel(const __grid_constant__ CUtensorMap tmK,
                           const __grid_constant__ CUtensorMap tmV,
                           const __nv_bfloat16* __restrict__ q, float* __restrict__ o_part,
                           float* __restrict__ lse_part, uint8_t* __restrict__ skip_mask,
                           int* __restrict__ status, int Hq, int Hkv, int L, int split_len,
-                          int n_splits, float scale_log2, float tau_log2, int tau_is_inf,
+                          int n_splits, float scale_log2, float tau_log2,
                           unsigned long long wait_limit_ns, int withhold_v,
                           const int* __restrict__ block_table, const int* __restrict__ seq_lens,
                           int max_pages) {
@@ -425,10 +427,10 @@ __global__ void __launch_bounds__(kDecThreads, (G <= 4) ? 2 : 1)
       // row lane % G passes iff it has a history and the tile max is below m - tau
       const bool pass =
           lane >= n_dec || (m_exact != NEG_INF && (mt == NEG_INF || mt < m_exact - tau_log2));
-      keep_i = tau_is_inf || !__all_sync(FULL, pass);
+      keep_i = !SKIP || !__all_sync(FULL, pass);
       // per-head rule: bit r set iff row r computes this tile (lanes 0..G-1 hold rows 0..G-1)
       unsigned row_keep = 0xffffffffu;
-      if constexpr (per_head) row_keep = tau_is_inf ? 0xffffffffu : __ballot_sync(FULL, !pass);
+      if constexpr (per_head && SKIP) row_keep = __ballot_sync(FULL, !pass);
       m_exact = fmaxf(m_exact, mt);  // a skipped tile never raises it
       if (keep_i) {
         const bool moved = m_exact > m_ref + kRefSlack;
@@ -674,10 +676,10 @@ bool dec_map(CUtensorMap* m, const void* base, int BH, int L, int D) {
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int D, int G, int RULE, bool PAGED>
+template <int D, int G, int RULE, bool PAGED, bool SKIP>
 int launch_dgrp(const DecodeLaunch& a) {
   using C = DecCfg<D, G>;
-  auto kern = decode_partial_kernel<D, G, RULE, PAGED>;
+  auto kern = decode_partial_kernel<D, G, RULE, PAGED, SKIP>;
   constexpr int smem_bytes = PAGED ? C::kSmemBytesPaged : C::kSmemBytes;
   static uint64_t attr_done = 0;
   int dev = 0;
@@ -700,7 +702,7 @@ int launch_dgrp(const DecodeLaunch& a) {
   kern<<<grid, kDecThreads, smem_bytes, a.stream>>>(
       mk, mv, static_cast<const __nv_bfloat16*>(a.q), a.o_part, a.lse_part, a.skip_mask,
       a.status, a.Hq, a.Hkv, a.L, a.split_len, a.n_splits, a.scale_log2, a.tau_log2,
-      a.tau_is_inf, a.wait_limit_ns, a.withhold_v, a.block_table, a.seq_lens, a.max_pages);
+      a.wait_limit_ns, a.withhold_v, a.block_table, a.seq_lens, a.max_pages);
   if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   decode_combine_kernel<D><<<a.B * a.Hq, D, 0, a.stream>>>(
       a.o_part, a.lse_part, static_cast<__nv_bfloat16*>(a.o), a.n_splits);
@@ -709,7 +711,9 @@ int launch_dgrp(const DecodeLaunch& a) {
 
 template <int D, int G, int RULE>
 int launch_dgr(const DecodeLaunch& a) {
-  return a.block_table ? launch_dgrp<D, G, RULE, true>(a) : launch_dgrp<D, G, RULE, false>(a);
+  if (a.tau_is_inf)
+    return a.block_table ? launch_dgrp<D, G, RULE, true, false>(a) : launch_dgrp<D, G, RULE, false, false>(a);
+  return a.block_table ? launch_dgrp<D, G, RULE, true, true>(a) : launch_dgrp<D, G, RULE, false, true>(a);
 }
 
 template <int D, int G>
