@@ -60,11 +60,9 @@ constexpr float kRescale = 8.0f;  // lazy rescale threshold (log2 units)
 // Which of the 16 column pairs of each 32-column chunk take the polynomial
 // exp2 instead of MUFU (bit c = pair c).  Measured on B200 the softmax here is
 // not bound by MUFU throughput, and every fraction tried (1/4 to 3/4) made
-// the kernel slower, so the default is none.
-#ifndef BSS_POLY_PAIRS
-#define BSS_POLY_PAIRS 0x0000u
-#endif
-constexpr uint32_t kPolyPairs = BSS_POLY_PAIRS;
+// this kernel slower, so it takes none; the column-split kernel offers the
+// polynomial through attn_prefill_poly.
+constexpr uint32_t kPolyPairs = 0x0000u;
 
 
 
@@ -1229,14 +1227,11 @@ int launch_prefill_pp(const PrefillLaunch& a) {
     }
     return ATTN_ERR_INVALID_ARG;
   }
-#ifndef BSS_PREFILL_SPLIT
-#define BSS_PREFILL_SPLIT 1
-#endif
   // d = Bc = 128, fixed length: the column-split kernel (three S buffers
   // beside one O accumulator; measured faster than two row blocks per CTA,
   // whose one S buffer per row block serialises S, softmax and P*V).  Bc = 64
   // keeps two row blocks per CTA with two S buffers each, measured faster.
-  if (BSS_PREFILL_SPLIT && a.d == 128 && a.Bc == 128 && !a.cu_seqlens) return launch_prefill_split(a);
+  if (a.d == 128 && a.Bc == 128 && !a.cu_seqlens) return launch_prefill_split(a);
   if (a.d == 128) return a.Bc == 64 ? pp_launch_c<128, 64>(a) : pp_launch_c<128, 128>(a);
   if (a.d == 64) return a.Bc == 64 ? pp_launch_c<64, 64>(a) : pp_launch_c<64, 128>(a);
   return ATTN_ERR_INVALID_ARG;
