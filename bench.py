@@ -422,8 +422,9 @@ def main():
                 "algorithmic_bytes": compulsory_prefill_bytes(wh),
                 "peak_source": f"{peak_src} bf16 burst; the sustained figure (seconds-long GEMM loop "
                                f"under the power cap) is given beside it",
-                "kernel": "prefill_split_kernel<128,causal> (one 128-row block per work item, softmax "
-                          "warpgroups splitting each key tile's columns, persistent)",
+                "kernel": "prefill_split_kernel<128, causal, no poly, no skip test> (tau = inf; one "
+                          "128-row block per work item, softmax warpgroups splitting each key tile's "
+                          "columns, persistent)",
                 "algorithmic": "2*B*Hq*N^2*d dense-equivalent FLOPs per launch (causal half of 4*N^2*d "
                                "per head); one launch per step"}
     configs[HEADLINE]["runs"].append(
